@@ -1,0 +1,170 @@
+"""Pins for the oracle's scale layouts, its GEMM and the pages' byte counts."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_block_scaled_10_b200 import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------------------- layouts
+
+def _pad(s, rmul, cmul):
+    R, C = s.shape
+    Rp, Cp = -(-R // rmul) * rmul, -(-C // cmul) * cmul
+    out = np.zeros((Rp, Cp), np.uint8)
+    out[:R, :C] = s
+    return out
+
+
+def _swz128_by_reshape(s):
+    """The 128x4 block-scale layout as a reshape/transpose: row = 128a + 32b + c,
+    column = 4d + e  ->  byte order [a][d][c][b][e]."""
+    p = _pad(s, 128, 4)
+    Rp, Cp = p.shape
+    return p.reshape(Rp // 128, 4, 32, Cp // 4, 4).transpose(0, 3, 2, 1, 4).reshape(-1)
+
+
+def _swz8_by_reshape(s):
+    """The 8x4 layout: row = 8a + b, column = 4c + d  ->  byte order [a][c][b][d]."""
+    p = _pad(s, 8, 4)
+    Rp, Cp = p.shape
+    return p.reshape(Rp // 8, 8, Cp // 4, 4).transpose(0, 2, 1, 3).reshape(-1)
+
+
+SHAPES = [(1, 1), (16, 32), (128, 4), (130, 7), (300, 33), (8, 448), (33, 512)]
+
+
+@pytest.mark.parametrize("R,C", SHAPES)
+def test_swizzle_128x4_matches_reshape(orc, R, C):
+    s = workloads.random_bytes((R, C), seed=R * 1000 + C, low=1, high=255)
+    got = orc.swizzle(s, orc.L128x4)
+    assert np.array_equal(got, _swz128_by_reshape(s))
+    assert np.array_equal(orc.unswizzle(got, R, C, orc.L128x4), s)
+
+
+@pytest.mark.parametrize("R,C", SHAPES)
+def test_swizzle_8x4_matches_reshape(orc, R, C):
+    s = workloads.random_bytes((R, C), seed=R * 1000 + C + 7, low=1, high=255)
+    got = orc.swizzle(s, orc.L8x4)
+    assert np.array_equal(got, _swz8_by_reshape(s))
+    assert np.array_equal(orc.unswizzle(got, R, C, orc.L8x4), s)
+
+
+@pytest.mark.parametrize("layout", [1, 2])
+def test_offsets_are_a_bijection_and_padding_is_zero(orc, layout):
+    R, C = 131, 9
+    nbytes = orc.sf_bytes(layout, R, C)
+    Rp = -(-R // (128 if layout == 1 else 8)) * (128 if layout == 1 else 8)
+    Cp = -(-C // 4) * 4
+    offs = sorted(orc.sf_offset(layout, r, c, R, C) for r in range(Rp) for c in range(Cp))
+    assert offs == list(range(nbytes))
+    s = np.full((R, C), 0xFF, np.uint8)
+    buf = orc.swizzle(s, layout)
+    assert int((buf == 0xFF).sum()) == R * C and int((buf == 0).sum()) == nbytes - R * C
+
+
+def test_sf_bytes_at_workload_shapes(orc):
+    assert orc.sf_bytes(orc.L128x4, 16, 512 // 16) == 4096
+    assert orc.sf_bytes(orc.L8x4, 16, 512 // 16) == 512
+    assert orc.sf_bytes(orc.L128x4, 8192, 7168 // 16) == 3670016
+    assert orc.sf_bytes(orc.L128x4, 4096, 14336 // 16) == 3670016
+    assert orc.sf_bytes(orc.L128x4, 28672, 8192 // 16) == 14680064
+    assert orc.sf_bytes(orc.L8x4, 1, 8192 // 16) == 8 * 512
+    assert orc.sf_bytes(orc.L128x4, 1, 8192 // 16) == 128 * 512
+
+
+# ------------------------------------------------------------------------------- GEMM
+
+E2M1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6])
+
+
+def _deq_numpy(q, sf, g):
+    vals = np.stack([E2M1[q & 0xF], E2M1[q >> 4]], axis=-1).reshape(q.shape[0], -1)
+    s = torch.from_numpy(np.ascontiguousarray(sf)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return vals * np.repeat(s, 16, axis=1) / np.float64(np.float32(g))
+
+
+def test_gemm_ones_gives_k(orc):
+    M, N, K = 3, 5, 256
+    a = np.full((M, K // 2), 0x22, np.uint8)  # both nibbles = E2M1 1.0
+    w = np.full((N, K // 2), 0x22, np.uint8)
+    sa = np.full((M, K // 16), 0x38, np.uint8)  # E4M3 1.0
+    sw = np.full((N, K // 16), 0x38, np.uint8)
+    out16, out64 = orc.gemm(a, sa, 1.0, w, sw, 1.0, want_f64=True)
+    assert (out64 == K).all()
+    assert (out16.view(np.float16) == K).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 16), (3, 5, 64), (8, 16, 128), (7, 3, 96), (16, 256, 512)])
+def test_gemm_brute_force_vs_numpy(orc, M, N, K):
+    seed = M * 100 + N * 10 + K
+    a = workloads.random_bytes((M, K // 2), seed)
+    w = workloads.random_bytes((N, K // 2), seed + 1)
+    sa = workloads.random_bytes((M, K // 16), seed + 2, 0x20, 0x50)
+    sw = workloads.random_bytes((N, K // 16), seed + 3, 0x20, 0x50)
+    ga, gw = 37.5, 1234.0
+    out16, out64 = orc.gemm(a, sa, ga, w, sw, gw, want_f64=True)
+    want = _deq_numpy(a, sa, ga) @ _deq_numpy(w, sw, gw).T
+    np.testing.assert_allclose(out64, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+    assert np.array_equal(out16, out64.astype(np.float16).view(np.uint16))
+
+
+def test_gemm_is_not_transposed(orc):
+    # A row 0 is all 1.0 and W row 1 is all 2.0, everything else zero: only D[0,1] != 0
+    K = 64
+    a = np.zeros((2, K // 2), np.uint8)
+    w = np.zeros((3, K // 2), np.uint8)
+    a[0, :] = 0x22
+    w[1, :] = 0x44
+    s1 = lambda r: np.full((r, K // 16), 0x38, np.uint8)
+    out = orc.gemm(a, s1(2), 1.0, w, s1(3), 1.0).view(np.float16)
+    want = np.zeros((2, 3), np.float16)
+    want[0, 1] = 2 * K
+    assert np.array_equal(out, want)
+
+
+def test_gemm_global_scales_divide(orc):
+    K = 32
+    a = np.full((1, K // 2), 0x22, np.uint8)
+    w = np.full((1, K // 2), 0x22, np.uint8)
+    s = np.full((1, K // 16), 0x38, np.uint8)
+    out16, out64 = orc.gemm(a, s, 4.0, w, s, 0.5, want_f64=True)
+    assert out64[0, 0] == K / (4.0 * 0.5)
+
+
+# ------------------------------------------------------------------------------- byte counts
+
+def _traffic_golden():
+    vals = {}
+    with open(os.path.join(GOLDEN, "swiglu_fp8_traffic.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                k, v = line.split()
+                vals[k] = float(v)
+    return vals
+
+
+def test_page_byte_counts_follow_from_printed_steps(orc):
+    gold = _traffic_golden()
+    N, H = 1, 1
+    unfused, fused, red = orc.swiglu_quant_traffic_as_printed(N, H)
+    assert unfused == gold["unfused_total"] == gold["unfused_read_x"] + gold["unfused_write_y_bf16"] + \
+        gold["unfused_read_y_bf16"] + gold["unfused_write_q_fp8"]
+    assert fused == gold["fused_total"] == gold["fused_read_x"] + gold["fused_write_q_fp8"]
+    assert round(100 * red) == round(100 * 4 / 13) == 31 and int(100 * red) == gold["reduction_percent"]
+
+
+def test_byte_counts_from_shapes(orc):
+    N, H = 4096, 14336
+    NH = N * H
+    u8, f8 = orc.swiglu_quant_traffic_from_shapes(N, H, "fp8")
+    assert (u8, f8) == (9 * NH, 5 * NH)
+    u4, f4 = orc.swiglu_quant_traffic_from_shapes(N, H, "nvfp4")
+    assert f4 == 4 * NH + NH // 2 + NH // 16 == 267911168
+    # the fused SwiGLU + NVFP4 workload moves 4.5625 NH bytes
+    assert f4 / NH == 4.5625
