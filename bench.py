@@ -1,0 +1,514 @@
+"""Benchmark of the NVFP4 hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload per_token|swiglu|decode|prefill|tiny] [--m 32] [--a-layout 128x4|8x4]
+
+Default workload: per-token NVFP4 quantize of X bf16 [8192, 7168] (N(0,1) with 0.1% of
+entries x50), one fp32 global scale per token, E4M3 scales in the 128x4 layout. A step is
+one call of the path on one batch; inputs are resident in HBM and rotated over enough
+copies that no step finds its input in the 126 MB L2.
+
+Prints one JSON line (rank 0). `value` is whole-job throughput in the workload's unit
+(GB/s of algorithmic bytes for the quantize kernels, TFLOP/s for the GEMMs), measured with
+CUDA events on the launching stream, max over ranks. Multi-GPU runs are independent
+replicas (weak scaling): the path has no exchange step.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 GEMM TFLOPS + quantize GB/s, each as % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0  # nominal dense ratio (9 PF fp4 / 2.25 PF bf16)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def algorithmic(workload, M=None, K=None, N=None, H=None, a_layout="128x4"):
+    """Algorithmic bytes (and FLOPs) of one launch: every input byte read once, every output
+    byte written once."""
+    if workload == "per_token":
+        x = M * K * 2
+        q = M * K // 2
+        sf = (-(-M // 128) * 128) * (-(-(K // 16) // 4) * 4)
+        g = M * 4
+        return {"bytes": x + q + sf + g, "read": x, "written": q + sf + g, "flops": 0}
+    if workload == "swiglu":
+        x = M * 2 * H * 2
+        q = M * H // 2
+        sf = (-(-M // 128) * 128) * (-(-(H // 16) // 4) * 4)
+        return {"bytes": x + q + sf, "read": x, "written": q + sf, "flops": 0}
+    if workload in ("decode", "prefill", "tiny"):
+        rows_a = (-(-M // 8) * 8) if a_layout == "8x4" else (-(-M // 128) * 128)
+        a = M * K // 2 + rows_a * K // 16
+        w = N * K // 2 + (-(-N // 128) * 128) * K // 16
+        out = M * N * 2
+        return {"bytes": a + w + out, "read": a + w, "written": out, "flops": 2 * M * N * K}
+    raise ValueError(workload)
+
+
+class Clocks:
+    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.bus_id = bus_id
+        self.proc = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.bus_id:
+            cmd += ["-i", self.bus_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
+                          and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def _source_hash(*rel):
+    h = hashlib.sha256()
+    for r in rel:
+        with open(os.path.join(ROOT, r), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu capture, if the kernel source still matches."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e:
+        return None
+    if e.get("source_sha") != _source_hash(*e["sources"]):
+        return None
+    return e["bytes_per_launch"]
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, torch, dist):
+    import nvfp4_block_scaled_10_b200 as nv
+    from nvfp4_block_scaled_10_b200 import build, workloads
+
+    build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    wl = args.workload
+    layout_code = nv.SF_8x4 if args.a_layout == "8x4" else nv.SF_128x4
+
+    # ---- inputs (resident in HBM, rotated so no step reuses L2-resident data)
+    if wl == "per_token":
+        M, K = 8192, 7168
+        x_host = workloads.per_token(M, K, seed=workloads.SEEDS["per_token"] + rank)
+        copies = [x_host.to(dev) for _ in range(3)]
+        g = torch.empty(M, dtype=torch.float32, device=dev)
+        q = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+        sf = torch.empty(nv.nvfp4_sf_bytes(M, K, nv.SF_128x4), dtype=torch.uint8, device=dev)
+        alg = algorithmic(wl, M=M, K=K)
+        kernel_key, kernel_name = "quant_pertoken_rowcache", "quant_pertoken_rowcache_kernel"
+
+        def step(i):
+            nv.nvfp4_quantize(copies[i % 3], g, per_token=True, sf_layout=nv.SF_128x4, q=q, sf=sf)
+        launches_per_step = 1
+        workload_desc = {"workload": "per-token NVFP4 quantize", "shape": [M, K], "input": "bf16",
+                         "dist": "N(0,1), 0.1% of entries x50", "scales": "E4M3 128x4",
+                         "global_scale": "fp32 per token", "l2": "input rotated over 3 copies (352 MB > 126 MB L2)"}
+        unit, factor = "GB/s", alg["bytes"] / 1e9
+    elif wl == "swiglu":
+        M, H = 4096, 14336
+        x_host = workloads.swiglu(M, H, seed=workloads.SEEDS["swiglu"] + rank)
+        copies = [x_host.to(dev) for _ in range(2)]
+        gval = 2688.0 / 60.0  # encode scale of |Y| up to ~60; value only, not a timing input
+        gdev = torch.tensor([gval], dtype=torch.float32, device=dev)
+        q = torch.empty(M, H // 2, dtype=torch.uint8, device=dev)
+        sf = torch.empty(nv.nvfp4_sf_bytes(M, H, nv.SF_128x4), dtype=torch.uint8, device=dev)
+        alg = algorithmic(wl, M=M, H=H)
+        kernel_key, kernel_name = "swiglu_quant", "swiglu_quant_kernel"
+
+        def step(i):
+            nv.swiglu_nvfp4_quantize(copies[i % 2], gdev, sf_layout=nv.SF_128x4, q=q, sf=sf)
+        launches_per_step = 1
+        workload_desc = {"workload": "fused SwiGLU + NVFP4 quantize", "shape": [M, 2 * H],
+                         "input": "bf16", "dist": "N(0,1)", "scales": "E4M3 128x4",
+                         "global_scale": "fp32 per tensor", "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
+        unit, factor = "GB/s", alg["bytes"] / 1e9
+    elif wl in ("decode", "prefill", "tiny"):
+        if wl == "decode":
+            M, N, K = args.m, 28672, 8192
+            a_b, w_b = workloads.decode(M, N, K)
+            ncopy = 2
+        elif wl == "prefill":
+            M = N = K = 8192
+            a_b, w_b = workloads.prefill()
+            ncopy = 3
+        else:
+            a_b, w_b = workloads.tiny()
+            M, K = a_b.shape
+            N = w_b.shape[0]
+            ncopy = 1
+        a_d, w_d = a_b.to(dev), w_b.to(dev)
+        ga = nv.nvfp4_global_scale(a_d)
+        gw = nv.nvfp4_global_scale(w_d)
+        ops = []
+        for _ in range(ncopy):
+            aq, asf, _ = nv.nvfp4_quantize(a_d, ga, sf_layout=layout_code)
+            wq, wsf, _ = nv.nvfp4_quantize(w_d, gw, sf_layout=nv.SF_128x4)
+            ops.append((aq, asf, wq, wsf))
+        del a_d, w_d
+        out = torch.empty(M, N, dtype=torch.float16, device=dev)
+        alg = algorithmic(wl, M=M, N=N, K=K, a_layout=args.a_layout)
+        kernel_key, kernel_name = f"gemm_{wl}", "gemm_nvfp4_kernel"
+
+        def step(i):
+            aq, asf, wq, wsf = ops[i % ncopy]
+            nv.nvfp4_gemm(aq, asf, ga, wq, wsf, gw, a_layout=layout_code, out=out)
+        launches_per_step = 1
+        workload_desc = {"workload": f"NVFP4 GEMM ({wl})", "M": M, "N": N, "K": K,
+                         "a_scales": args.a_layout, "w_scales": "128x4", "out": "fp16",
+                         "l2": f"operands rotated over {ncopy} copies"}
+        if wl == "decode":
+            unit, factor = "GB/s", alg["bytes"] / 1e9
+        else:
+            unit, factor = "TFLOP/s", alg["flops"] / 1e12
+    else:
+        raise SystemExit(f"unknown workload {wl}")
+
+    torch.cuda.synchronize()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, per-launch events on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+    except Exception:
+        bus = None
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with Clocks(bus if rank == 0 else None) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(args.warmup + i)
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    total_ms = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in ev]
+    if dist is not None:
+        tt = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = tt.item()
+    ms_per_step = total_ms / args.steps
+    value = world * factor / (total_ms / 1e3 / args.steps)
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if wl in ("per_token", "swiglu"):
+        src = copies[0]
+        h_in = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
+        h_in.copy_(src.cpu())
+        h_q = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        h_sf = torch.empty(sf.shape, dtype=sf.dtype, pin_memory=True)
+        h_g = torch.empty(g.shape, dtype=g.dtype, pin_memory=True) if wl == "per_token" else None
+        d_in = torch.empty_like(src)
+
+        def e2e_step():
+            d_in.copy_(h_in, non_blocking=True)
+            if wl == "per_token":
+                nv.nvfp4_quantize(d_in, g, per_token=True, sf_layout=nv.SF_128x4, q=q, sf=sf)
+                h_g.copy_(g, non_blocking=True)
+            else:
+                nv.swiglu_nvfp4_quantize(d_in, gdev, sf_layout=nv.SF_128x4, q=q, sf=sf)
+            h_q.copy_(q, non_blocking=True)
+            h_sf.copy_(sf, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if dist is not None:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = tt.item()
+        d2h = h_q.numel() + h_sf.numel() + (h_g.numel() * 4 if h_g is not None else 0)
+        e2e = {"value": world * factor / (e2e_ms / 1e3), "unit": unit,
+               "h2d_bytes_per_step": h_in.numel() * 2, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms}
+    elif wl in ("decode", "prefill", "tiny"):
+        aq, asf, wq, wsf = ops[0]
+        hs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (aq, asf, wq, wsf)]
+        for h, t in zip(hs, (aq, asf, wq, wsf)):
+            h.copy_(t.cpu())
+        ds = [torch.empty_like(t) for t in (aq, asf, wq, wsf)]
+        h_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+
+        def e2e_step():
+            for d, h in zip(ds, hs):
+                d.copy_(h, non_blocking=True)
+            nv.nvfp4_gemm(ds[0], ds[1], ga, ds[2], ds[3], gw, a_layout=layout_code, out=out)
+            h_out.copy_(out, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = 3
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if dist is not None:
+            tt = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = tt.item()
+        e2e = {"value": world * factor / (e2e_ms / 1e3), "unit": unit,
+               "h2d_bytes_per_step": sum(h.numel() for h in hs), "d2h_bytes_per_step": h_out.numel() * 2,
+               "ms_per_step": e2e_ms}
+
+    # ---- roofline of the dominant kernel (the only kernel of the step)
+    pk, pk_kind = peaks()
+    launch_avg = statistics.mean(launch_ms)
+    if unit == "GB/s":
+        achieved = alg["bytes"] / 1e9 / (launch_avg / 1e3)
+        peak = float(pk["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "peak_source": f"{pk_kind} hbm_gbs (copy)"}
+    else:
+        achieved = alg["flops"] / 1e12 / (launch_avg / 1e3)
+        peak = float(pk["bf16_tflops"]) * FP4_OVER_BF16
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak,
+                "peak_source": f"{pk_kind} bf16_tflops (burst) x {FP4_OVER_BF16:g} nominal fp4/bf16 ratio"}
+    roof["traffic"] = recorded_traffic(kernel_key)
+    roof["algorithmic_bytes_per_launch"] = alg["bytes"]
+    roof["kernel"] = kernel_name
+    roof["launch_ms"] = launch_avg
+
+    result = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {**workload_desc, "parallelism": f"replicas x{world}"},
+        "roofline": roof, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary() if rank == 0 else None,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(wl, args)
+    return result
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def _oracle_sample(wl, args):
+    """A bounded sample of the same workload for the oracle: returns (callable, units, desc)."""
+    import numpy as np
+
+    import oracle
+    from nvfp4_block_scaled_10_b200 import workloads
+
+    if wl == "per_token":
+        rows = args.cpu_rows
+        x = workloads.per_token(8192, 7168)
+        bits = workloads.bits16(x[:rows])
+        alg = algorithmic("per_token", M=rows, K=7168)
+        return (lambda: oracle.quantize(bits, oracle.BF16, per_token=True)), alg["bytes"] / 1e9, \
+            f"first {rows} of 8192 rows", "GB/s"
+    if wl == "swiglu":
+        rows = max(1, args.cpu_rows // 2)
+        x = workloads.swiglu(rows, 14336)
+        bits = workloads.bits16(x)
+        g = 2688.0 / 60.0
+        alg = algorithmic("swiglu", M=rows, H=14336)
+        return (lambda: oracle.swiglu_quantize(bits, g, oracle.BF16)), alg["bytes"] / 1e9, \
+            f"{rows} of 4096 rows", "GB/s"
+    if wl in ("decode", "prefill", "tiny"):
+        if wl == "decode":
+            M, N, K = args.m, 512, 8192
+            a, w = workloads.decode(args.m, 28672, 8192)
+            w = w[:N]
+            desc = f"M={args.m}, 512 of 28672 weight rows"
+        elif wl == "prefill":
+            M, N, K = 64, 1024, 8192
+            a, w = workloads.prefill()
+            a, w = a[:M], w[:N]
+            desc = "64 of 8192 rows x 1024 of 8192 columns"
+        else:
+            a, w = workloads.tiny()
+            M, K = a.shape
+            N = w.shape[0]
+            desc = "full"
+        ab, wb = workloads.bits16(a), workloads.bits16(w)
+        ga, gw = oracle.global_scale(ab), oracle.global_scale(wb)
+        aq, sa, _ = oracle.quantize(ab, g=ga)
+        wq, sw, _ = oracle.quantize(wb, g=gw)
+        if wl == "decode":
+            alg = algorithmic("decode", M=M, N=N, K=K)
+            return (lambda: oracle.gemm(aq, sa, ga, wq, sw, gw)), alg["bytes"] / 1e9, desc, "GB/s"
+        return (lambda: oracle.gemm(aq, sa, ga, wq, sw, gw)), 2 * M * N * K / 1e12, desc, "TFLOP/s"
+    raise ValueError(wl)
+
+
+def _threads_used():
+    # the oracle is single-threaded C; numpy's fp64 matmul may use BLAS threads
+    try:
+        from threadpoolctl import threadpool_info
+        n = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        n = 1
+    return n
+
+
+def cpu_baseline(wl, args):
+    fn, units, desc, unit = _oracle_sample(wl, args)
+    t = time.perf_counter()
+    fn()
+    dt = time.perf_counter() - t
+    cores = 1 if wl in ("per_token", "swiglu") else _threads_used()
+    return {"value": units / dt, "unit": unit, "cores": cores, "kind": "oracle",
+            "sample": desc, "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    fn, units, desc, unit = _oracle_sample(args.workload, args)
+    for _ in range(args.warmup):
+        fn()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        fn()
+    dt = (time.perf_counter() - t) / args.steps
+    cores = 1 if args.workload in ("per_token", "swiglu") else _threads_used()
+    value = units / dt
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "sample": desc, "runs": "CPU oracle (plain C)"},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="per_token",
+                    choices=["per_token", "swiglu", "decode", "prefill", "tiny"])
+    ap.add_argument("--m", type=int, default=32, help="tokens of the decode workload")
+    ap.add_argument("--a-layout", default="128x4", choices=["128x4", "8x4"])
+    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist_mod
+
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_mod
+    try:
+        res = run_ours(args, rank, world, torch, dist)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

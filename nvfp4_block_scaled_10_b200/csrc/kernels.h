@@ -1,0 +1,51 @@
+// kernels.h -- internal declarations shared by the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+namespace nvfp4 {
+
+constexpr int kSfLinear = 0;
+constexpr int kSf128x4 = 1;
+constexpr int kSf8x4 = 2;
+constexpr int kInBf16 = 0;
+constexpr int kInFp16 = 1;
+
+constexpr int kRowcacheMaxStages = 6;
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s without progress
+constexpr int kDevErrTimeout = 1;
+
+// quantize.cu
+int *device_error_symbol();
+int global_scale_parts(int64_t M, int64_t K, int num_sms);
+cudaError_t launch_global_scale(const void *x, int dtype, int64_t M, int64_t K, int64_t ldx,
+                                float *g_out, float *partial, int nparts, cudaStream_t st);
+cudaError_t launch_quantize(const void *x, int dtype, int64_t M, int64_t K, int64_t ldx, float *g,
+                            int per_token, uint8_t *q, uint8_t *sf, int layout, int64_t Rp,
+                            int64_t Cp, int num_sms, int max_smem_optin, cudaStream_t st);
+cudaError_t launch_swiglu_quantize(const void *x, int dtype, int64_t M, int64_t H, int64_t ldx,
+                                   const float *g, uint8_t *q, uint8_t *sf, int layout, int64_t Rp,
+                                   int64_t Cp, int num_sms, cudaStream_t st);
+cudaError_t launch_sf_swizzle(const uint8_t *lin, uint8_t *out, int64_t R, int64_t C, int layout,
+                              int64_t Rp, int64_t Cp, int num_sms, cudaStream_t st);
+cudaError_t launch_sf_unswizzle(const uint8_t *in, uint8_t *lin, int64_t R, int64_t C, int layout,
+                                int64_t Cp, int num_sms, cudaStream_t st);
+
+// gemm_sm100.cu
+struct GemmArgs {
+  const uint8_t *a_q;
+  const uint8_t *a_sf;
+  int a_layout;
+  const float *a_g;
+  const uint8_t *w_q;
+  const uint8_t *w_sf;
+  const float *w_g;
+  void *out;
+  int64_t M, N, K;
+  int32_t *dev_status;
+};
+cudaError_t launch_gemm(const GemmArgs &args, int num_sms, cudaStream_t st);
+
+}  // namespace nvfp4

@@ -77,6 +77,7 @@ def lib():
             "orc_sf_swizzle": (None, [vp, i64, i64, i32, vp]),
             "orc_sf_unswizzle": (None, [vp, i64, i64, i32, vp]),
             "orc_gemm": (None, [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, vp]),
+            "orc_dequantize": (None, [vp, vp, f32, i64, i64, vp]),
             "orc_e2m1_encode_array": (None, [vp, i64, vp]),
             "orc_e4m3_encode_array": (None, [vp, i64, vp]),
             "orc_exp_array": (None, [vp, i64, vp]),
@@ -261,12 +262,34 @@ def unswizzle(buf: np.ndarray, R: int, C: int, layout: int) -> np.ndarray:
 
 # ----------------------------------------------------------------------------- GEMM
 
+def dequantize(q, sf_lin, g) -> np.ndarray:
+    """fp64 values E2M1(q) * E4M3(s) / g of a packed operand [rows, K/2]."""
+    qq = _c(q, np.uint8)
+    ss = _c(sf_lin, np.uint8)
+    rows, K2 = qq.shape
+    K = 2 * K2
+    assert ss.shape == (rows, K // 16)
+    out = np.zeros((rows, K), np.float64)
+    lib().orc_dequantize(_p(qq), _p(ss), float(np.float32(g)), rows, K, _p(out))
+    return out
+
+
 def gemm(a_q, a_sf_lin, a_g, w_q, w_sf_lin, w_g, want_f64: bool = False):
-    """D = fp16_rn(sum_k deq(a)[m,k] deq(w)[n,k]), fp64 sum.
+    """D = fp16_rn(deq(A) @ deq(W)^T): dequantization in the C oracle, the fp64 product by
+    numpy's matmul (a library step), one rounding to fp16 by the C oracle.
 
     a_q [M,K/2], a_sf_lin [M,K/16], w_q [N,K/2], w_sf_lin [N,K/16]; g's are scalars.
     Returns fp16 bits [M,N] (uint16), plus the fp64 sums when want_f64.
     """
+    da = dequantize(a_q, a_sf_lin, a_g)
+    dw = dequantize(w_q, w_sf_lin, w_g)
+    out64 = np.matmul(da, dw.T)
+    out16 = f64_to_f16(out64.reshape(-1)).reshape(out64.shape)
+    return (out16, out64) if want_f64 else out16
+
+
+def gemm_loops(a_q, a_sf_lin, a_g, w_q, w_sf_lin, w_g, want_f64: bool = False):
+    """The same GEMM as three plain loops in C (fp64 sum in k order); for tiny shapes."""
     a = _c(a_q, np.uint8)
     w = _c(w_q, np.uint8)
     sa = _c(a_sf_lin, np.uint8)

@@ -441,6 +441,18 @@ void orc_gemm(const uint8_t *a, const uint8_t *sa, float ga, const uint8_t *w, c
     }
 }
 
+/*
+ * Dequantize a packed operand: out[r, k] = E2M1(q[r, k]) * E4M3(s[r, k/16]) / g in fp64
+ * (the same expression the loop GEMM above uses for each factor).
+ */
+void orc_dequantize(const uint8_t *q, const uint8_t *s, float g, int64_t rows, int64_t K,
+                    double *out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t k = 0; k < K; ++k)
+      out[r * K + k] =
+          elem_value(q + r * (K / 2), k) * orc_e4m3_value(s[r * (K / 16) + k / 16]) / (double)g;
+}
+
 /* ------------------------------------------------------------------------------------ */
 /* Array helpers for the pin tests (elementwise loops over the scalar definitions).       */
 /* ------------------------------------------------------------------------------------ */

@@ -1,0 +1,118 @@
+"""GPU parity of the block-scaled FP4 GEMM against the oracle (fp64 sum, one fp16 rounding).
+
+Tolerance (normwise and elementwise, see helpers.gemm_close): 1e-3 of the result. Small
+shapes cover swap-AB decode tiles, ragged M/N/K tails and both activation-scale layouts; the
+decode and prefill workloads are checked at full size on sampled outputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from nvfp4_block_scaled_10_b200 import workloads
+from tests.helpers import gemm_close, host_bytes, require_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def _random_operands(M, N, K, seed):
+    a = workloads.random_bytes((M, K // 2), seed)
+    w = workloads.random_bytes((N, K // 2), seed + 1)
+    sa = workloads.random_bytes((M, K // 16), seed + 2, 0x28, 0x48)
+    sw = workloads.random_bytes((N, K // 16), seed + 3, 0x28, 0x48)
+    return a, sa, 3.5, w, sw, 250.0
+
+
+def _quantized_operands(a_bf16, w_bf16):
+    ab, wb = workloads.bits16(a_bf16), workloads.bits16(w_bf16)
+    ga = orc.global_scale(ab)
+    gw = orc.global_scale(wb)
+    a, sa, _ = orc.quantize(ab, g=ga)
+    w, sw, _ = orc.quantize(wb, g=gw)
+    return a, sa, ga, w, sw, gw
+
+
+def _to_device(nv, a, sa, ga, w, sw, gw, a_layout):
+    return dict(
+        a_q=torch.from_numpy(a).cuda(),
+        a_sf=torch.from_numpy(orc.swizzle(sa, a_layout)).cuda(),
+        a_g=torch.tensor([ga], dtype=torch.float32, device="cuda"),
+        w_q=torch.from_numpy(w).cuda(),
+        w_sf=torch.from_numpy(orc.swizzle(sw, orc.L128x4)).cuda(),
+        w_g=torch.tensor([gw], dtype=torch.float32, device="cuda"),
+        a_layout=a_layout,
+    )
+
+
+def _run(nv, ops, a_layout):
+    dev = _to_device(nv, *ops, a_layout)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = nv.nvfp4_gemm(**dev, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    return out.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+SMALL = [(1, 256, 512), (8, 256, 512), (16, 256, 512), (32, 512, 1024), (3, 136, 64),
+         (33, 256, 512), (128, 256, 256), (130, 520, 320), (256, 1024, 2048), (300, 264, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", SMALL)
+def test_gemm_parity_small(M, N, K):
+    nv = require_cuda()
+    ops = _random_operands(M, N, K, seed=M * 1000 + N + K)
+    _, ref = orc.gemm(*ops, want_f64=True)
+    layouts = [orc.L128x4, orc.L8x4] if M <= 32 else [orc.L128x4]
+    for layout in layouts:
+        got = _run(nv, ops, layout)
+        gemm_close(got, ref)
+
+
+def test_gemm_tiny_workload():
+    """A [16,512] ~N(0,1), W [256,512] ~N(0,0.02) quantized by the oracle; both layouts."""
+    nv = require_cuda()
+    a, w = workloads.tiny()
+    ops = _quantized_operands(a, w)
+    _, ref = orc.gemm(*ops, want_f64=True)
+    for layout in (orc.L128x4, orc.L8x4):
+        gemm_close(_run(nv, ops, layout), ref)
+
+
+@pytest.fixture(scope="module")
+def decode_weights():
+    _, w = workloads.decode(1)
+    wb = workloads.bits16(w)
+    gw = orc.global_scale(wb)
+    wq, ws, _ = orc.quantize(wb, g=gw)
+    return wq, ws, gw
+
+
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_gemm_decode_workload(decode_weights, M):
+    """W NVFP4 [28672, 8192], A NVFP4 [M, 8192]; both activation-scale layouts; 512 sampled
+    output columns (weight rows) against the oracle."""
+    nv = require_cuda()
+    wq, ws, gw = decode_weights
+    a_bf16, _ = workloads.decode(M, N=16, K=8192)  # the activation draw of this workload
+    ab = workloads.bits16(a_bf16)
+    ga = orc.global_scale(ab)
+    aq, sa, _ = orc.quantize(ab, g=ga)
+    cols = np.sort(np.random.default_rng(M).choice(wq.shape[0], 512, replace=False))
+    _, ref = orc.gemm(aq, sa, ga, wq[cols], ws[cols], gw, want_f64=True)
+    for layout in (orc.L128x4, orc.L8x4):
+        got = _run(nv, (aq, sa, ga, wq, ws, gw), layout)
+        gemm_close(got[:, cols], ref)
+
+
+def test_gemm_prefill_workload():
+    """A, W NVFP4 [8192, 8192] from bf16 N(0,1) / N(0,0.02); 24 sampled rows x 1024 columns."""
+    nv = require_cuda()
+    a, w = workloads.prefill()
+    ops = _quantized_operands(a, w)
+    got = _run(nv, ops, orc.L128x4)
+    aq, sa, ga, wq, ws, gw = ops
+    rng = np.random.default_rng(7)
+    rows = np.sort(np.concatenate([[0, 127, 128, 8191], rng.choice(8192, 20, replace=False)]))
+    cols = np.sort(np.concatenate([[0, 255, 256, 8191], rng.choice(8192, 1020, replace=False)]))
+    _, ref = orc.gemm(aq[rows], sa[rows], ga, wq[cols], ws[cols], gw, want_f64=True)
+    gemm_close(got[np.ix_(rows, cols)], ref)
+    assert np.isfinite(got.view(np.float16)).all()

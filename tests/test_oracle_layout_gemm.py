@@ -94,23 +94,46 @@ def test_gemm_ones_gives_k(orc):
     w = np.full((N, K // 2), 0x22, np.uint8)
     sa = np.full((M, K // 16), 0x38, np.uint8)  # E4M3 1.0
     sw = np.full((N, K // 16), 0x38, np.uint8)
-    out16, out64 = orc.gemm(a, sa, 1.0, w, sw, 1.0, want_f64=True)
-    assert (out64 == K).all()
-    assert (out16.view(np.float16) == K).all()
+    for fn in (orc.gemm, orc.gemm_loops):
+        out16, out64 = fn(a, sa, 1.0, w, sw, 1.0, want_f64=True)
+        assert (out64 == K).all()
+        assert (out16.view(np.float16) == K).all()
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 1, 16), (3, 5, 64), (8, 16, 128), (7, 3, 96), (16, 256, 512)])
-def test_gemm_brute_force_vs_numpy(orc, M, N, K):
+def test_gemm_loops_brute_force_vs_numpy(orc, M, N, K):
     seed = M * 100 + N * 10 + K
     a = workloads.random_bytes((M, K // 2), seed)
     w = workloads.random_bytes((N, K // 2), seed + 1)
     sa = workloads.random_bytes((M, K // 16), seed + 2, 0x20, 0x50)
     sw = workloads.random_bytes((N, K // 16), seed + 3, 0x20, 0x50)
     ga, gw = 37.5, 1234.0
-    out16, out64 = orc.gemm(a, sa, ga, w, sw, gw, want_f64=True)
+    out16, out64 = orc.gemm_loops(a, sa, ga, w, sw, gw, want_f64=True)
     want = _deq_numpy(a, sa, ga) @ _deq_numpy(w, sw, gw).T
     np.testing.assert_allclose(out64, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
     assert np.array_equal(out16, out64.astype(np.float16).view(np.uint16))
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 5, 64), (16, 256, 512), (33, 70, 1024)])
+def test_gemm_matmul_path_equals_loops(orc, M, N, K):
+    # the fast oracle (C dequantize + fp64 matmul) against the plain triple loop
+    seed = M * 7 + N * 3 + K
+    a = workloads.random_bytes((M, K // 2), seed)
+    w = workloads.random_bytes((N, K // 2), seed + 1)
+    sa = workloads.random_bytes((M, K // 16), seed + 2, 0x20, 0x50)
+    sw = workloads.random_bytes((N, K // 16), seed + 3, 0x20, 0x50)
+    l16, l64 = orc.gemm_loops(a, sa, 3.0, w, sw, 700.0, want_f64=True)
+    m16, m64 = orc.gemm(a, sa, 3.0, w, sw, 700.0, want_f64=True)
+    np.testing.assert_allclose(m64, l64, rtol=1e-12, atol=1e-12 * np.abs(l64).max())
+    diff = np.abs(m16.view(np.float16).astype(np.float64) - l16.view(np.float16).astype(np.float64))
+    ulp = np.abs(l16.view(np.float16).astype(np.float64)) * 2.0 ** -10 + 2.0 ** -24
+    assert (diff <= ulp).all()
+
+
+def test_dequantize_matches_independent_decode(orc):
+    q = workloads.random_bytes((5, 32), 9)
+    s = workloads.random_bytes((5, 4), 10, 0, 0x7F)
+    assert np.array_equal(orc.dequantize(q, s, 2.5), _deq_numpy(q, s, 2.5))
 
 
 def test_gemm_is_not_transposed(orc):
@@ -121,10 +144,10 @@ def test_gemm_is_not_transposed(orc):
     a[0, :] = 0x22
     w[1, :] = 0x44
     s1 = lambda r: np.full((r, K // 16), 0x38, np.uint8)
-    out = orc.gemm(a, s1(2), 1.0, w, s1(3), 1.0).view(np.float16)
     want = np.zeros((2, 3), np.float16)
     want[0, 1] = 2 * K
-    assert np.array_equal(out, want)
+    for fn in (orc.gemm, orc.gemm_loops):
+        assert np.array_equal(fn(a, s1(2), 1.0, w, s1(3), 1.0).view(np.float16), want)
 
 
 def test_gemm_global_scales_divide(orc):
@@ -132,8 +155,9 @@ def test_gemm_global_scales_divide(orc):
     a = np.full((1, K // 2), 0x22, np.uint8)
     w = np.full((1, K // 2), 0x22, np.uint8)
     s = np.full((1, K // 16), 0x38, np.uint8)
-    out16, out64 = orc.gemm(a, s, 4.0, w, s, 0.5, want_f64=True)
-    assert out64[0, 0] == K / (4.0 * 0.5)
+    for fn in (orc.gemm, orc.gemm_loops):
+        out16, out64 = fn(a, s, 4.0, w, s, 0.5, want_f64=True)
+        assert out64[0, 0] == K / (4.0 * 0.5)
 
 
 # ------------------------------------------------------------------------------- byte counts

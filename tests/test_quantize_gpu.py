@@ -1,0 +1,218 @@
+"""GPU parity of the quantize kernels against the oracle: bit-exact bytes.
+
+Small shapes span several CTAs, ragged tails and every layout; the full per-token and
+SwiGLU workloads are compared in full."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+from nvfp4_block_scaled_10_b200 import workloads
+from tests.helpers import assert_bytes_equal, host_bytes, require_cuda, to_dev_bits
+
+pytestmark = pytest.mark.gpu
+
+DT = {"bf16": (torch.bfloat16, orc.BF16), "fp16": (torch.float16, orc.FP16)}
+
+
+def _inputs(M, K, pad, seed, dtype):
+    x = workloads.with_outliers((M, K + pad), seed=seed, dtype=DT[dtype][0])
+    return x
+
+
+def _quantize_both(nv, xt, dtype, per_token, layout, K):
+    """Runs GPU and oracle on the same bits (x may have a row stride > K)."""
+    tdt, odt = DT[dtype]
+    xs = xt[:, :K]
+    bits = workloads.bits16(xs.contiguous())
+    M = xs.shape[0]
+    xd = xt.cuda()[:, :K]
+    if per_token:
+        g_dev = torch.full((M,), -1.0, dtype=torch.float32, device="cuda")
+        q_o, sf_o, g_o = orc.quantize(bits, odt, per_token=True)
+    else:
+        g = orc.global_scale(bits, odt)
+        g_dev = torch.tensor([g], dtype=torch.float32, device="cuda")
+        q_o, sf_o, g_o = orc.quantize(bits, odt, g=g)
+    sf_dev = torch.full((nv.nvfp4_sf_bytes(M, K, layout),), 0xAA, dtype=torch.uint8, device="cuda")
+    q_dev = torch.full((M, K // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    nv.nvfp4_quantize(xd, g_dev, per_token=per_token, sf_layout=layout, q=q_dev, sf=sf_dev)
+    torch.cuda.synchronize()
+    assert_bytes_equal(host_bytes(q_dev), q_o, "q")
+    assert_bytes_equal(host_bytes(sf_dev), orc.swizzle(sf_o, layout), "sf")
+    if per_token:
+        assert_bytes_equal(host_bytes(g_dev), g_o.view(np.uint8), "g")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("per_token", [False, True])
+@pytest.mark.parametrize("layout", [0, 1, 2])
+@pytest.mark.parametrize("M,K,pad", [(1, 16, 0), (3, 48, 8), (17, 512, 0), (130, 1040, 16),
+                                     (257, 64, 0), (300, 7168, 0)])
+def test_quantize_parity_small(M, K, pad, layout, per_token, dtype):
+    nv = require_cuda()
+    xt = _inputs(M, K, pad, seed=M * 31 + K, dtype=dtype)
+    _quantize_both(nv, xt, dtype, per_token, layout, K)
+
+
+def test_quantize_per_token_long_rows_two_pass():
+    # rows of 65536 elements (128 KB) do not fit twice in shared memory: two-pass path
+    nv = require_cuda()
+    xt = _inputs(3, 65536, 0, seed=5, dtype="bf16")
+    _quantize_both(nv, xt, "bf16", True, 1, 65536)
+
+
+def test_quantize_worked_blocks_and_edges():
+    nv = require_cuda()
+    # hand-derived blocks (ties, saturation after scale rounding, zeros, -0) as GPU input
+    rows = []
+    with open(__file__.replace("test_quantize_gpu.py", "golden/quant_worked_blocks.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                parts = [p.strip() for p in line.split("|")]
+                rows.append((float(parts[1]), [float(v) for v in parts[2].split()]))
+    for g, xs in rows:
+        x = torch.tensor([xs], dtype=torch.float32).to(torch.bfloat16)
+        bits = workloads.bits16(x)
+        q_o, sf_o, _ = orc.quantize(bits, orc.BF16, g=g)
+        q, sf, _ = nv.nvfp4_quantize(x.cuda(), torch.tensor([g], device="cuda"),
+                                     sf_layout=nv.SF_LINEAR)
+        torch.cuda.synchronize()
+        assert_bytes_equal(host_bytes(q), q_o, f"q g={g} {xs}")
+        assert_bytes_equal(host_bytes(sf), sf_o, f"sf g={g} {xs}")
+    # tiny negatives (-> -0 codes), exact zeros, a huge g (scale overflow -> saturation)
+    x = torch.tensor([[-1e-3, -0.0, 0.0, 1e-3] * 4, [65000.0] + [-1e-30] * 15],
+                     dtype=torch.float32).to(torch.bfloat16)
+    for g in [1.0, 2688.0, 3.0e38]:
+        bits = workloads.bits16(x)
+        q_o, sf_o, _ = orc.quantize(bits, orc.BF16, g=g)
+        q, sf, _ = nv.nvfp4_quantize(x.cuda(), torch.tensor([g], device="cuda"),
+                                     sf_layout=nv.SF_LINEAR)
+        torch.cuda.synchronize()
+        assert_bytes_equal(host_bytes(q), q_o, f"q g={g}")
+        assert_bytes_equal(host_bytes(sf), sf_o, f"sf g={g}")
+
+
+def test_quantize_empty_is_noop():
+    nv = require_cuda()
+    x = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    q, sf, g = nv.nvfp4_quantize(x, per_token=True)
+    assert q.numel() == 0 and g.numel() == 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("M,K,pad", [(1, 16, 0), (16, 512, 0), (256, 512, 0), (77, 1040, 24),
+                                     (1000, 4096, 0)])
+def test_global_scale_parity(M, K, pad, dtype):
+    nv = require_cuda()
+    xt = _inputs(M, K, pad, seed=M + K + pad, dtype=dtype)
+    bits = workloads.bits16(xt[:, :K].contiguous())
+    g_o = orc.global_scale(bits, DT[dtype][1])
+    g = nv.nvfp4_global_scale(xt.cuda()[:, :K])
+    torch.cuda.synchronize()
+    assert g.item() == g_o
+
+
+def test_global_scale_zero_tensor():
+    nv = require_cuda()
+    g = nv.nvfp4_global_scale(torch.zeros(5, 32, dtype=torch.bfloat16, device="cuda"))
+    assert g.item() == 1.0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("layout", [0, 1, 2])
+@pytest.mark.parametrize("M,H,pad", [(1, 16, 0), (5, 48, 8), (33, 512, 0), (130, 1024, 16),
+                                     (64, 14336, 0)])
+def test_swiglu_parity_small(M, H, pad, layout, dtype):
+    nv = require_cuda()
+    tdt, odt = DT[dtype]
+    xt = workloads.normal((M, 2 * H + pad), 1.0, seed=M * 13 + H, dtype=tdt)
+    xs = xt[:, :2 * H].contiguous()
+    bits = workloads.bits16(xs)
+    g = orc.global_scale_from_amax(orc.swiglu_amax(bits, odt))
+    q_o, sf_o = orc.swiglu_quantize(bits, g, odt)
+    sf_dev = torch.full((nv.nvfp4_sf_bytes(M, H, layout),), 0xAA, dtype=torch.uint8, device="cuda")
+    q, sf = nv.swiglu_nvfp4_quantize(xt.cuda()[:, :2 * H], torch.tensor([g], device="cuda"),
+                                     sf_layout=layout, sf=sf_dev)
+    torch.cuda.synchronize()
+    assert_bytes_equal(host_bytes(q), q_o, "q")
+    assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, layout), "sf")
+
+
+def test_swiglu_extreme_gates():
+    nv = require_cuda()
+    # gates far outside the exp clamp range and around zero
+    gate = torch.tensor([[-200.0, -90.0, -88.5, -87.5, -20.0, -1e-3, 0.0, 1e-3, 0.5, 1.0,
+                          20.0, 87.0, 88.5, 200.0, -5.0, 5.0]], dtype=torch.float32)
+    up = torch.linspace(-3, 3, 16).reshape(1, 16)
+    x = torch.cat([gate, up], dim=1).to(torch.bfloat16)
+    bits = workloads.bits16(x)
+    for g in [1.0, 100.0]:
+        q_o, sf_o = orc.swiglu_quantize(bits, g, orc.BF16)
+        q, sf = nv.swiglu_nvfp4_quantize(x.cuda(), torch.tensor([g], device="cuda"),
+                                         sf_layout=nv.SF_LINEAR)
+        torch.cuda.synchronize()
+        assert_bytes_equal(host_bytes(q), q_o, "q")
+        assert_bytes_equal(host_bytes(sf), sf_o, "sf")
+
+
+@pytest.mark.parametrize("layout", [0, 1, 2])
+@pytest.mark.parametrize("R,C", [(1, 1), (130, 7), (300, 33), (28672, 512)])
+def test_swizzle_unswizzle_parity(R, C, layout):
+    nv = require_cuda()
+    lin = workloads.random_bytes((R, C), seed=R + C + layout, low=1, high=255)
+    want = orc.swizzle(lin, layout)
+    out = torch.full((want.size,), 0xAA, dtype=torch.uint8, device="cuda")
+    got = nv.nvfp4_sf_swizzle(torch.from_numpy(lin).cuda(), layout, out=out)
+    back = nv.nvfp4_sf_unswizzle(got, R, C, layout)
+    torch.cuda.synchronize()
+    assert_bytes_equal(host_bytes(got), want, "swizzle")
+    assert_bytes_equal(host_bytes(back), lin, "unswizzle")
+
+
+# ------------------------------------------------------------------------------ full size
+
+def test_per_token_workload_full():
+    """[8192, 7168] bf16 with 0.1% x50 outliers, per-token g, 128x4 scales: every byte."""
+    nv = require_cuda()
+    x = workloads.per_token()
+    bits = workloads.bits16(x)
+    q_o, sf_o, g_o = orc.quantize(bits, orc.BF16, per_token=True)
+    q, sf, g = nv.nvfp4_quantize(x.cuda(), per_token=True, sf_layout=nv.SF_128x4)
+    torch.cuda.synchronize()
+    assert_bytes_equal(host_bytes(g), g_o.view(np.uint8), "g")
+    assert_bytes_equal(host_bytes(q), q_o, "q")
+    assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, orc.L128x4), "sf")
+
+
+def test_swiglu_workload_full():
+    """[4096, 2 x 14336] bf16, per-tensor g from amax(Y) by the oracle, 128x4: every byte."""
+    nv = require_cuda()
+    x = workloads.swiglu()
+    bits = workloads.bits16(x)
+    g = orc.global_scale_from_amax(orc.swiglu_amax(bits, orc.BF16))
+    q_o, sf_o = orc.swiglu_quantize(bits, g, orc.BF16)
+    q, sf = nv.swiglu_nvfp4_quantize(x.cuda(), torch.tensor([g], device="cuda"),
+                                     sf_layout=nv.SF_128x4)
+    torch.cuda.synchronize()
+    assert_bytes_equal(host_bytes(q), q_o, "q")
+    assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, orc.L128x4), "sf")
+
+
+def test_tiny_workload_quantize():
+    """A [16,512] and W [256,512], per-tensor g from the GPU amax kernel, both layouts."""
+    nv = require_cuda()
+    a, w = workloads.tiny()
+    for t in (a, w):
+        bits = workloads.bits16(t)
+        g_o = orc.global_scale(bits, orc.BF16)
+        g = nv.nvfp4_global_scale(t.cuda())
+        torch.cuda.synchronize()
+        assert g.item() == g_o
+        q_o, sf_o, _ = orc.quantize(bits, orc.BF16, g=g_o)
+        for layout in (nv.SF_128x4, nv.SF_8x4):
+            q, sf, _ = nv.nvfp4_quantize(t.cuda(), g, sf_layout=layout)
+            torch.cuda.synchronize()
+            assert_bytes_equal(host_bytes(q), q_o, "q")
+            assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, layout), "sf")
