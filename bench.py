@@ -235,9 +235,9 @@ def run_ours(args, rank, world, torch, dist):
     # ---- timed region: K steps, per-launch events on the launching stream
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    bus = None
     try:
-        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        pr = torch.cuda.get_device_properties(dev)
+        bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
     except Exception:
         bus = None
     if dist is not None:
