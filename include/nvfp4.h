@@ -46,7 +46,8 @@ typedef enum {
   NVFP4_ERR_MISALIGNED = 2,  /* a pointer or leading dimension breaks the 16-byte rule */
   NVFP4_ERR_UNSUPPORTED = 3, /* valid but outside what this build implements */
   NVFP4_ERR_CUDA = 4,        /* a CUDA runtime/driver call or a launch failed */
-  NVFP4_ERR_TIMEOUT = 5      /* a bounded device wait gave up (see nvfp4_gemm dev_status) */
+  NVFP4_ERR_TIMEOUT = 5,     /* a bounded device wait gave up (see nvfp4_gemm dev_status) */
+  NVFP4_ERR_SCRATCH_LIMIT = 6 /* input larger than a fixed library scratch array covers */
 } nvfp4_status;
 
 /* Block-scale buffer layouts. For R rows and C = K/16 scale columns:
@@ -100,6 +101,25 @@ NVFP4_API size_t nvfp4_global_scale_workspace_bytes(int64_t M, int64_t K);
  */
 NVFP4_API int nvfp4_global_scale(const void *x, int dtype, int64_t M, int64_t K, int64_t ldx, float *g_out,
                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * nvfp4_global_scale without a workspace argument, for callers that cannot allocate device
+ * memory where they call it: an engine's enqueue() that is handed tensor pointers but no
+ * allocator, or a runtime with a fixed memory plan that must not cudaMalloc/cudaFree per
+ * call (both synchronize the device and can fail under memory pressure mid-request). The
+ * pages have no counterpart to this entry point; it computes the same g as
+ * nvfp4_global_scale (bit-identical result) from the same arguments minus the workspace.
+ * The reduction scratch is a 16 KB array inside the library, one per device, kept until the
+ * process exits. The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress) and the SM count; make that first call before any stream capture.
+ * Limit: M * K <= 2^28 elements (268,435,456); larger inputs return
+ * NVFP4_ERR_SCRATCH_LIMIT and enqueue nothing. All calls on a device share the array:
+ * calls whose kernels may overlap on the GPU (unordered streams) race and can return a
+ * wrong g -- order them on one stream. Allocates nothing.
+ * Requires: x 16-byte aligned, K % 16 == 0, ldx % 8 == 0, ldx >= K, g_out 4-byte aligned.
+ */
+NVFP4_API int nvfp4_global_scale_noalloc(const void *x, int dtype, int64_t M, int64_t K,
+                                         int64_t ldx, float *g_out, void *stream);
 
 /*
  * NVFP4 quantize ("perf: optimize per-token nvfp4 quantization kernel", FlashInfer PR

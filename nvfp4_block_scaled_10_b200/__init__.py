@@ -19,7 +19,7 @@ import torch
 SF_LINEAR, SF_128x4, SF_8x4 = 0, 1, 2
 IN_BF16, IN_FP16 = 0, 1
 
-OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_MISALIGNED, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = range(7)
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libnvfp4.so")
 
@@ -30,6 +30,7 @@ SIGNATURES = {
     "nvfp4_sf_bytes": (_i64, [_i64, _i64, _i32]),
     "nvfp4_global_scale_workspace_bytes": (_sz, [_i64, _i64]),
     "nvfp4_global_scale": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "nvfp4_global_scale_noalloc": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _vp]),
     "swiglu_nvfp4_quantize": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp]),
     "nvfp4_sf_swizzle": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
@@ -120,6 +121,18 @@ def nvfp4_global_scale(x: torch.Tensor, g_out: torch.Tensor | None = None,
     _check(lib().nvfp4_global_scale(_ptr(x), _dtype_code(x), M, K, ldx, _ptr(g_out),
                                     _ptr(workspace), workspace.numel(), _stream(stream)),
            "nvfp4_global_scale")
+    return g_out
+
+
+def nvfp4_global_scale_noalloc(x: torch.Tensor, g_out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Same g as nvfp4_global_scale, reduction scratch inside the library (no workspace).
+
+    For callers that cannot allocate at the call site; `g_out` (device fp32 [1]) is theirs.
+    Inputs above 2^28 elements raise (NVFP4_ERR_SCRATCH_LIMIT).
+    """
+    M, K, ldx = _rows_ld(x)
+    _check(lib().nvfp4_global_scale_noalloc(_ptr(x), _dtype_code(x), M, K, ldx, _ptr(g_out),
+                                            _stream(stream)), "nvfp4_global_scale_noalloc")
     return g_out
 
 

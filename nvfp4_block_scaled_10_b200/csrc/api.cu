@@ -83,6 +83,7 @@ const char *nvfp4_status_str(int status) {
     case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED";
     case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
     case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT";
+    case NVFP4_ERR_SCRATCH_LIMIT: return "NVFP4_ERR_SCRATCH_LIMIT";
     default: return "NVFP4_ERR_UNKNOWN";
   }
 }
