@@ -8,16 +8,28 @@
 // weight scale; output FP16 [B,N]. The AllReduce that plugin appends is not part of this
 // kernel.
 //
-// Structure (one output tile per CTA, 192 threads):
-//   warp 0      TMA producer: 2-D tiled copies of the packed operands (128-byte swizzle) and
-//               bulk copies of the 512-byte scale atoms into a STAGES-deep shared-memory ring.
-//   warp 1      allocates TMEM; one lane issues tcgen05.cp (scales -> TMEM) and
-//               tcgen05.mma.kind::mxf4nvf4.block_scale (MMA K = 64) into an fp32 TMEM
-//               accumulator, and tcgen05.commit to release ring slots.
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one TMEM lane quarter per warp),
-//               scale by 1 / (ga * gw), round to fp16, store.
+// Persistent, warp-specialised kernel (one CTA per SM, tiles handed out round-robin):
+//   warp 0        TMA producer: 2-D tiled copies of the packed operands (128-byte swizzle)
+//                 and bulk copies of the 512-byte scale atoms into a STAGES-deep ring.
+//   warp 1        allocates TMEM; one lane issues tcgen05.mma.kind::mxf4nvf4.block_scale
+//                 (MMA K = 64) into an fp32 TMEM accumulator and tcgen05.commit.
+//   warps 4..7    scale warps: warp 4+q moves the scale words that TMEM lane quarter q needs
+//                 from the shared-memory atoms into TMEM with tcgen05.st, one TMEM scale slot
+//                 per ring stage (tcgen05.cp copies of whole atoms cost about as much tensor
+//                 pipe time as the MMAs; tcgen05.st from other warps does not slow them).
+//   warps 8..     epilogue: tcgen05.ld of the accumulator (lane quarter = warp % 4), scale
+//                 by 1 / (ga * gw) and round to fp16 in registers, release the accumulator,
+//                 then store.
+//
+// Scale layout the MMA reads (measured on B200 with probes): TMEM lane quarter q (lanes
+// 32 q .. 32 q + 31, accumulator rows 32 q .. 32 q + 31) reads both operands' scales from its
+// own lanes. A row m = 32 q + i: the 32-bit word (four E4M3 scales of one K64 step) at lane
+// m, column base + q. B row n: lane 32 q + n % 32, column base + n / 32, so B's scales are
+// replicated into all four quarters. Bases are column-aligned (4 columns per K64 step, 8 for
+// a 256-row B operand); an unaligned base raised a misaligned-address error.
+//
 // Small M (decode): the operands swap roles (weights are the MMA's 128-row A operand, the
-// tokens its N = BN columns) so the weight stream, not the token count, fills the MMA.
+// tokens its N = BN columns) so the weight stream fills the MMA.
 #include <cfloat>
 #include <cstdint>
 
@@ -30,11 +42,12 @@
 
 namespace nvfp4 {
 
-constexpr int kBM = 128;        // MMA M: rows of the A operand per tile
-constexpr int kBKBytes = 128;   // packed bytes of K per stage (256 FP4 elements)
-constexpr int kK64PerStage = 4; // MMA K is 64 elements (32 bytes)
+constexpr int kBM = 128;           // MMA M: rows of the A operand per tile
+constexpr int kBKBytes = 128;      // packed bytes of K per stage (256 FP4 elements)
+constexpr int kK64PerStage = 4;    // MMA K is 64 elements (32 bytes)
 constexpr int kSfAtomBytes = 512;  // 128 rows x 4 scales (the 128x4 atom)
-constexpr int kThreads = 192;
+constexpr int kSfWarp0 = 4;        // first scale warp
+constexpr int kEpiWarp0 = 8;       // first epilogue warp
 
 template <int BN, int STAGES, bool SWAP>
 struct Cfg {
@@ -49,21 +62,28 @@ struct Cfg {
   static constexpr int kOffSfa = kOffB + STAGES * kBBytes;
   static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
   static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
-  static constexpr int kBarBytes = (2 * STAGES + 1) * 8 + 8;
+  static constexpr int kAccBufs = BN <= 128 ? 2 : 1;
+  // full[S], empty[S], sf_full[S], acc_full[A], acc_empty[A], tmem slot
+  static constexpr int kBarBytes = (3 * STAGES + 2 * kAccBufs) * 8 + 16;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;  // + alignment slack
-  // TMEM columns: accumulator [0, BN) (at least 32), then A scales, then B scales
+  // TMEM columns: accumulators, then per stage one scale slot (A scales, then B scales)
   static constexpr int kAccCols = BN < 32 ? 32 : BN;
-  static constexpr int kSfaCol = kAccCols;
-  static constexpr int kSfaCols = 4 * kK64PerStage;
-  static constexpr int kSfbCol = kSfaCol + kSfaCols;
-  static constexpr int kSfbCols = 4 * kSfbBlocks * kK64PerStage;
-  static constexpr int kUsedCols = kSfbCol + kSfbCols;
+  static constexpr int kSfaColsPerK64 = 4;
+  static constexpr int kSfbColsPerK64 = BN > 128 ? 8 : 4;
+  static constexpr int kSlotCols = kK64PerStage * (kSfaColsPerK64 + kSfbColsPerK64);
+  static constexpr int kSfCol0 = kAccBufs * kAccCols;
+  static constexpr int kUsedCols = kSfCol0 + STAGES * kSlotCols;
   static constexpr int kTmemCols = kUsedCols <= 32    ? 32
                                    : kUsedCols <= 64  ? 64
                                    : kUsedCols <= 128 ? 128
                                    : kUsedCols <= 256 ? 256
                                                       : 512;
+  // epilogue: 8 warps (two per lane quarter, 128 columns each) for BN = 256, else 4
+  static constexpr int kEpiWarps = BN > 128 ? 8 : 4;
+  static constexpr int kColsPerEpiWarp = BN * 4 / kEpiWarps;
+  static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
   static_assert(BN % 8 == 0 && BN >= 8 && BN <= 256, "MMA N");
+  static_assert(kUsedCols <= 512, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
   // Instruction descriptor of tcgen05.mma.kind::mxf4nvf4: A and B are E2M1 (format 1),
   // K-major, dense, UE4M3 scales (bit 23 = 0), N >> 3 at bit 17, M >> 4 at bit 24.
@@ -79,23 +99,49 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
          (static_cast<uint64_t>(2) << 61);
 }
 
-// Descriptor of one 512-byte scale atom as the tcgen05.cp source: 32 rows of 16 bytes,
-// no swizzle, 8-row core matrices 128 bytes apart (SBO); one 16-byte column (LBO unused).
-__device__ __forceinline__ uint64_t desc_sf_atom(uint32_t saddr) {
-  return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(128 >> 4) << 32) |
-         (static_cast<uint64_t>(1) << 46);
+// 4 consecutive TMEM columns of this warp's 32 lanes, all set to v. The store takes a range
+// of four distinct registers, so the value is copied into four temporaries first (naming
+// one register four times leaves columns 1-3 with whatever the neighbouring registers hold).
+__device__ __forceinline__ void tmem_st_x4_rep(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "{\n\t.reg .b32 t0, t1, t2, t3;\n\t"
+      "mov.b32 t0, %1;\n\tmov.b32 t1, %1;\n\tmov.b32 t2, %1;\n\tmov.b32 t3, %1;\n\t"
+      "tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {t0, t1, t2, t3};\n\t}" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+// 4 consecutive TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st_x4(uint32_t taddr, uint32_t v0, uint32_t v1, uint32_t v2,
+                                           uint32_t v3) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+               "r"(v0), "r"(v1), "r"(v2), "r"(v3)
+               : "memory");
+}
+
+// 8 consecutive TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st_x8(uint32_t taddr, uint4 a, uint4 b) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+                   taddr),
+               "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 struct KernelParams {
   const uint8_t *sfa;  // scales of the MMA A operand (128x4 layout)
   const uint8_t *sfb;  // scales of the MMA B operand (128x4, or 8x4 when sfb_8x4)
   int sfb_8x4;
-  int64_t sfa_rows_padded;  // rows of the A-scale buffer
   int64_t sfb_rows_padded;  // rows of the B-scale buffer
   const float *ga;
   const float *gw;
   __half *out;
   int64_t M, N, K;  // problem shape in the caller's (unswapped) terms
+  int tiles_a;      // tiles along the MMA A operand (128 rows each)
+  int tiles_b;      // tiles along the MMA B operand (BN rows each)
   int32_t *dev_status;
 };
 
@@ -104,7 +150,7 @@ __device__ __forceinline__ void report_timeout(int32_t *dev_status) {
 }
 
 template <int BN, int STAGES, bool SWAP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a,
                       const __grid_constant__ CUtensorMap tmap_b, const KernelParams p) {
   using C = Cfg<BN, STAGES, SWAP>;
@@ -113,8 +159,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *empty = full + STAGES;
-  uint64_t *acc_full = empty + STAGES;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_full + 1);
+  uint64_t *sf_full = empty + STAGES;
+  uint64_t *acc_full = sf_full + STAGES;
+  uint64_t *acc_empty = acc_full + C::kAccBufs;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + C::kAccBufs);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -122,17 +170,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_k64 = static_cast<int>(K / 64);
   const int num_kt = (num_k64 + kK64PerStage - 1) / kK64PerStage;
   const int64_t k64_per_row = K / 64;  // 128x4 atoms per 128-row block
-
-  // tile origin: rows of the MMA A operand (a0) and of the MMA B operand (b0)
-  const int64_t a0 = static_cast<int64_t>(blockIdx.x) * kBM;
-  const int64_t b0 = static_cast<int64_t>(blockIdx.y) * BN;
+  const int num_tiles = p.tiles_a * p.tiles_b;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 4);  // one arrival per scale warp
     }
-    mbar_init(acc_full, 1);
+    for (int b = 0; b < C::kAccBufs; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], C::kEpiWarps);
+    }
     fence_mbar_init();
     prefetch_tmap(&tmap_a);
     prefetch_tmap(&tmap_b);
@@ -146,42 +195,51 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // Tile t covers MMA-A rows [a0, a0 + 128) and MMA-B rows [b0, b0 + BN).
+  auto tile_origin = [&](int t, int64_t &a0, int64_t &b0) {
+    a0 = static_cast<int64_t>(t % p.tiles_a) * kBM;
+    b0 = static_cast<int64_t>(t / p.tiles_a) * BN;
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    for (int kt = 0; kt < num_kt; ++kt) {
-      const int stage = kt % STAGES;
-      const int round = kt / STAGES;
-      if (kt >= STAGES) {
-        if (!mbar_wait_bounded(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
-          if (lane == 0) report_timeout(p.dev_status);
-          break;
-        }
-      }
-      const int k64_0 = kt * kK64PerStage;
-      const int nk64 = min(kK64PerStage, num_k64 - k64_0);
-      // scale bytes this stage brings by bulk copy
-      const int64_t sfa_block = a0 / 128;
-      uint32_t bytes = C::kABytes + C::kBBytes + nk64 * kSfAtomBytes;
+    uint32_t it = 0;  // ring position across tiles
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      int64_t a0, b0;
+      tile_origin(t, a0, b0);
       int sfb_copies = 0;
       if (!p.sfb_8x4) {
         for (int blk = 0; blk < C::kSfbBlocks; ++blk)
           if ((b0 / 128 + blk) * 128 < p.sfb_rows_padded) ++sfb_copies;
-        bytes += sfb_copies * nk64 * kSfAtomBytes;
       }
-      uint8_t *sA = smem + C::kOffA + stage * C::kABytes;
-      uint8_t *sB = smem + C::kOffB + stage * C::kBBytes;
-      uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
-      uint8_t *sSfb = smem + C::kOffSfb + stage * C::kSfbBytes;
-      if (lane == 0) {
-        asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(
-                         smem_u32(&full[stage])),
-                     "r"(bytes)
-                     : "memory");
-        tma_load_2d(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(a0), &full[stage]);
-        tma_load_2d(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(b0), &full[stage]);
-        bulk_g2s(sSfa, p.sfa + (sfa_block * k64_per_row + k64_0) * kSfAtomBytes,
-                 nk64 * kSfAtomBytes, &full[stage]);
-        if (!p.sfb_8x4) {
+      for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        const int stage = static_cast<int>(it % STAGES);
+        const uint32_t round = it / STAGES;
+        if (it >= STAGES) {
+          if (!mbar_wait_warp(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
+            if (lane == 0) report_timeout(p.dev_status);
+            ok = false;
+            break;
+          }
+        }
+        const int k64_0 = kt * kK64PerStage;
+        const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+        const uint32_t bytes = C::kABytes + C::kBBytes + nk64 * kSfAtomBytes +
+                               sfb_copies * nk64 * kSfAtomBytes;
+        uint8_t *sA = smem + C::kOffA + stage * C::kABytes;
+        uint8_t *sB = smem + C::kOffB + stage * C::kBBytes;
+        uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
+        uint8_t *sSfb = smem + C::kOffSfb + stage * C::kSfbBytes;
+        if (lane == 0) {
+          asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(
+                           smem_u32(&full[stage])),
+                       "r"(bytes)
+                       : "memory");
+          tma_load_2d(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(a0), &full[stage]);
+          tma_load_2d(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(b0), &full[stage]);
+          bulk_g2s(sSfa, p.sfa + ((a0 / 128) * k64_per_row + k64_0) * kSfAtomBytes,
+                   nk64 * kSfAtomBytes, &full[stage]);
           for (int blk = 0; blk < sfb_copies; ++blk) {
             const int64_t rb = b0 / 128 + blk;
             bulk_g2s(sSfb + blk * kK64PerStage * kSfAtomBytes,
@@ -189,115 +247,195 @@ __global__ void __launch_bounds__(kThreads, 1)
                      &full[stage]);
           }
         }
-      }
-      if (p.sfb_8x4) {
-        // 8x4 activation scales (BN <= 32 tokens): rebuild the 128x4 atom rows the TMEM copy
-        // expects. Lane r moves row r's 4 scales of each K64 step into bytes [16 r, 16 r + 4).
-        const int64_t r = lane;
-        for (int a = 0; a < nk64; ++a) {
-          uint32_t v = 0;
-          if (r < p.sfb_rows_padded && r < BN) {
-            v = *reinterpret_cast<const uint32_t *>(
-                p.sfb + ((r / 8) * k64_per_row + (k64_0 + a)) * 32 + (r % 8) * 4);
+        if (p.sfb_8x4) {
+          // 8x4 activation scales (BN <= 32 tokens): lane r puts row r's 4 scales of each K64
+          // step at bytes [16 r, 16 r + 4) of that step's atom, as a 128x4 atom has them.
+          const int64_t r = lane;
+          for (int a = 0; a < nk64; ++a) {
+            uint32_t v = 0;
+            if (r < p.sfb_rows_padded && r < BN) {
+              v = *reinterpret_cast<const uint32_t *>(
+                  p.sfb + ((r / 8) * k64_per_row + (k64_0 + a)) * 32 + (r % 8) * 4);
+            }
+            *reinterpret_cast<uint32_t *>(sSfb + a * kSfAtomBytes + r * 16) = v;
           }
-          *reinterpret_cast<uint32_t *>(sSfb + a * kSfAtomBytes + r * 16) = v;
         }
-        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&full[stage]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full[stage]);
+    }
+    // Tail: wait until the MMAs have released every stage still in use, so no tcgen05.commit
+    // arrival is outstanding when the CTA exits.
+    if (ok) {
+      const uint32_t used = it < STAGES ? it : STAGES;
+      for (uint32_t i = 0; i < used; ++i) {
+        const uint32_t j = it - used + i;
+        if (!mbar_wait_warp(&empty[j % STAGES], (j / STAGES) & 1, kWaitTimeoutNs)) {
+          if (lane == 0) report_timeout(p.dev_status);
+          break;
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      uint32_t it = 0;
+      uint32_t tile_iter = 0;
       bool ok = true;
-      for (int kt = 0; kt < num_kt; ++kt) {
-        const int stage = kt % STAGES;
-        const int round = kt / STAGES;
-        if (!mbar_wait_bounded(&full[stage], round & 1, kWaitTimeoutNs)) {
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tile_iter) {
+        const int buf = static_cast<int>(tile_iter % C::kAccBufs);
+        const uint32_t use = tile_iter / C::kAccBufs;
+        if (use > 0 && !mbar_wait_bounded(&acc_empty[buf], (use - 1) & 1, kWaitTimeoutNs)) {
           report_timeout(p.dev_status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * C::kAccCols;
+        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+          const int stage = static_cast<int>(it % STAGES);
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait_bounded(&full[stage], round & 1, kWaitTimeoutNs) ||
+              !mbar_wait_bounded(&sf_full[stage], round & 1, kWaitTimeoutNs)) {
+            report_timeout(p.dev_status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
+          const uint32_t sA = smem_u32(smem + C::kOffA + stage * C::kABytes);
+          const uint32_t sB = smem_u32(smem + C::kOffB + stage * C::kBBytes);
+          const uint32_t slot = tmem_base + C::kSfCol0 + stage * C::kSlotCols;
+          for (int a = 0; a < nk64; ++a) {
+            mma_nvf4(d_tmem, desc_sw128(sA + a * 32), desc_sw128(sB + a * 32), C::kIdesc,
+                     slot + a * C::kSfaColsPerK64,
+                     slot + kK64PerStage * C::kSfaColsPerK64 + a * C::kSfbColsPerK64,
+                     (kt | a) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[stage]);
+        }
+        if (ok) tc_commit(&acc_full[buf]);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kSfWarp0 && warp < kSfWarp0 + 4) {
+    // ------------------------------------------------------------------ scale warps
+    const int q = warp & 3;  // TMEM lane quarter this warp writes
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        const int stage = static_cast<int>(it % STAGES);
+        const uint32_t round = it / STAGES;
+        if (!mbar_wait_warp(&full[stage], round & 1, kWaitTimeoutNs)) {
+          if (lane == 0) report_timeout(p.dev_status);
           ok = false;
           break;
         }
         tc_fence_after();
         const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
-        const uint32_t sA = smem_u32(smem + C::kOffA + stage * C::kABytes);
-        const uint32_t sB = smem_u32(smem + C::kOffB + stage * C::kBBytes);
-        const uint32_t sSfa = smem_u32(smem + C::kOffSfa + stage * C::kSfaBytes);
-        const uint32_t sSfb = smem_u32(smem + C::kOffSfb + stage * C::kSfbBytes);
+        const uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
+        const uint8_t *sSfb = smem + C::kOffSfb + stage * C::kSfbBytes;
+        const uint32_t slot = lane_base + C::kSfCol0 + stage * C::kSlotCols;
+        const uint32_t slot_b = slot + kK64PerStage * C::kSfaColsPerK64;
+        // Each TMEM lane quarter q feeds accumulator rows 32 q .. 32 q + 31 and reads both
+        // operands' scales from its own 32 lanes: A row m = 32 q + lane at column
+        // (step base + q); B row n at lane 32 q + n % 32, column (step base + n / 32).
+        // Writing A's aligned 4-column group with the same word keeps the store aligned;
+        // B's scales are replicated into every quarter.
         for (int a = 0; a < nk64; ++a) {
-          tmem_cp_32x128b_x4(tmem_base + C::kSfaCol + 4 * a, desc_sf_atom(sSfa + a * kSfAtomBytes));
-          for (int blk = 0; blk < C::kSfbBlocks; ++blk)
-            tmem_cp_32x128b_x4(tmem_base + C::kSfbCol + (a * C::kSfbBlocks + blk) * 4,
-                               desc_sf_atom(sSfb + (blk * kK64PerStage + a) * kSfAtomBytes));
+          const uint32_t wa =
+              *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
+          tmem_st_x4_rep(slot + a * C::kSfaColsPerK64, wa);
+          // atom row `lane` holds B rows lane + 32 t' (t' = 0..3) of its 128-row block
+          const uint4 b0 = *reinterpret_cast<const uint4 *>(sSfb + a * kSfAtomBytes + lane * 16);
+          if constexpr (C::kSfbBlocks == 1) {
+            tmem_st_x4(slot_b + a * C::kSfbColsPerK64, b0.x, b0.y, b0.z, b0.w);
+          } else {
+            const uint4 b1 = *reinterpret_cast<const uint4 *>(
+                sSfb + (kK64PerStage + a) * kSfAtomBytes + lane * 16);
+            tmem_st_x8(slot_b + a * C::kSfbColsPerK64, b0, b1);
+          }
         }
-        for (int a = 0; a < nk64; ++a) {
-          mma_nvf4(tmem_base, desc_sw128(sA + a * 32), desc_sw128(sB + a * 32), C::kIdesc,
-                   tmem_base + C::kSfaCol + 4 * a,
-                   tmem_base + C::kSfbCol + a * C::kSfbBlocks * 4, (kt | a) != 0 ? 1u : 0u);
-        }
-        tc_commit(&empty[stage]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[stage]);
       }
-      if (ok) tc_commit(acc_full);
     }
-    __syncwarp();
-  } else {
+  } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int row = quarter * 32 + lane;
-    const bool ok = mbar_wait_bounded(acc_full, 0, kWaitTimeoutNs);
-    if (!ok) {
-      if (lane == 0) report_timeout(p.dev_status);
-    } else {
+    const int e = warp - kEpiWarp0;
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int col0 = (e / 4) * C::kColsPerEpiWarp;
+    const int row = q * 32 + lane;
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(p.ga[0], p.gw[0]));
+    uint32_t tile_iter = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_iter) {
+      int64_t a0, b0;
+      tile_origin(t, a0, b0);
+      const int buf = static_cast<int>(tile_iter % C::kAccBufs);
+      const uint32_t use = tile_iter / C::kAccBufs;
+      if (!mbar_wait_warp(&acc_full[buf], use & 1, kWaitTimeoutNs)) {
+        if (lane == 0) report_timeout(p.dev_status);
+        break;
+      }
       tc_fence_after();
-      const float alpha = __fdiv_rn(1.0f, __fmul_rn(p.ga[0], p.gw[0]));
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t t_acc =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols + col0;
       if constexpr (!SWAP) {
-        const int64_t m = a0 + row;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(t_row + c0, v);
-          tmem_wait_ld();
-          if (m < p.M) {
-            __half *dst = p.out + m * p.N + b0 + c0;
+        // fp16 pairs of this thread's row, columns [col0, col0 + kColsPerEpiWarp)
+        uint32_t h2[C::kColsPerEpiWarp / 2];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const int64_t n = b0 + c0 + 8 * j;
-              if (n + 8 <= p.N) {
-                uint4 pk;
-                __half2 h0 = __floats2half2_rn(__fmul_rn(__uint_as_float(v[8 * j + 0]), alpha),
-                                               __fmul_rn(__uint_as_float(v[8 * j + 1]), alpha));
-                __half2 h1 = __floats2half2_rn(__fmul_rn(__uint_as_float(v[8 * j + 2]), alpha),
-                                               __fmul_rn(__uint_as_float(v[8 * j + 3]), alpha));
-                __half2 h2 = __floats2half2_rn(__fmul_rn(__uint_as_float(v[8 * j + 4]), alpha),
-                                               __fmul_rn(__uint_as_float(v[8 * j + 5]), alpha));
-                __half2 h3 = __floats2half2_rn(__fmul_rn(__uint_as_float(v[8 * j + 6]), alpha),
-                                               __fmul_rn(__uint_as_float(v[8 * j + 7]), alpha));
-                pk.x = *reinterpret_cast<uint32_t *>(&h0);
-                pk.y = *reinterpret_cast<uint32_t *>(&h1);
-                pk.z = *reinterpret_cast<uint32_t *>(&h2);
-                pk.w = *reinterpret_cast<uint32_t *>(&h3);
-                *reinterpret_cast<uint4 *>(dst + 8 * j) = pk;
-              }
+        for (int c = 0; c < C::kColsPerEpiWarp; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t_acc + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            __half2 h = __floats2half2_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
+                                          __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
+            h2[c / 2 + j] = *reinterpret_cast<uint32_t *>(&h);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        const int64_t m = a0 + row;
+        if (m < p.M) {
+          __half *dst = p.out + m * p.N + b0 + col0;
+#pragma unroll
+          for (int j = 0; j < C::kColsPerEpiWarp / 8; ++j) {
+            if (b0 + col0 + 8 * j + 8 <= p.N) {
+              uint4 pk;
+              pk.x = h2[4 * j + 0];
+              pk.y = h2[4 * j + 1];
+              pk.z = h2[4 * j + 2];
+              pk.w = h2[4 * j + 3];
+              *reinterpret_cast<uint4 *>(dst + 8 * j) = pk;
             }
           }
         }
       } else {
         // accumulator lane = weight row n, column = token m
-        const int64_t n = a0 + row;
-#pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 8) {
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(t_row + c0, v);
-          tmem_wait_ld();
-          if (n < p.N) {
+        float vals[C::kColsPerEpiWarp];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int64_t m = b0 + c0 + j;
-              if (m < p.M)
-                p.out[m * p.N + n] = __float2half_rn(__fmul_rn(__uint_as_float(v[j]), alpha));
-            }
+        for (int c = 0; c < C::kColsPerEpiWarp; c += 8) {
+          uint32_t v[8];
+          tmem_ld_32x32b_x8(t_acc + c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) vals[c + j] = __fmul_rn(__uint_as_float(v[j]), alpha);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        const int64_t n = a0 + row;
+        if (n < p.N) {
+#pragma unroll
+          for (int j = 0; j < C::kColsPerEpiWarp; ++j) {
+            const int64_t m = b0 + col0 + j;
+            if (m < p.M) p.out[m * p.N + n] = __float2half_rn(vals[j]);
           }
         }
       }
@@ -349,7 +487,7 @@ static bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, i
 }
 
 template <int BN, int STAGES, bool SWAP>
-static cudaError_t run(const GemmArgs &g, cudaStream_t st) {
+static cudaError_t run(const GemmArgs &g, int num_sms, cudaStream_t st) {
   using C = Cfg<BN, STAGES, SWAP>;
   CUtensorMap ma, mb;
   KernelParams p{};
@@ -361,7 +499,6 @@ static cudaError_t run(const GemmArgs &g, cudaStream_t st) {
     p.sfa = g.a_sf;
     p.sfb = g.w_sf;
     p.sfb_8x4 = 0;
-    p.sfa_rows_padded = (g.M + 127) / 128 * 128;
     p.sfb_rows_padded = rows_sf_w;
   } else {
     if (!make_operand_map(&ma, g.w_q, g.N, kb, kBM)) return cudaErrorInvalidValue;
@@ -369,7 +506,6 @@ static cudaError_t run(const GemmArgs &g, cudaStream_t st) {
     p.sfa = g.w_sf;
     p.sfb = g.a_sf;
     p.sfb_8x4 = g.a_layout == kSf8x4 ? 1 : 0;
-    p.sfa_rows_padded = rows_sf_w;
     p.sfb_rows_padded = p.sfb_8x4 ? (g.M + 7) / 8 * 8 : (g.M + 127) / 128 * 128;
   }
   p.ga = g.a_g;
@@ -381,19 +517,20 @@ static cudaError_t run(const GemmArgs &g, cudaStream_t st) {
   p.dev_status = g.dev_status;
   const int64_t rows_a = SWAP ? g.N : g.M;
   const int64_t rows_b = SWAP ? g.M : g.N;
-  dim3 grid(static_cast<unsigned>((rows_a + kBM - 1) / kBM),
-            static_cast<unsigned>((rows_b + BN - 1) / BN));
+  p.tiles_a = static_cast<int>((rows_a + kBM - 1) / kBM);
+  p.tiles_b = static_cast<int>((rows_b + BN - 1) / BN);
+  const int64_t tiles = static_cast<int64_t>(p.tiles_a) * p.tiles_b;
+  const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<BN, STAGES, SWAP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  gemm_nvfp4_kernel<BN, STAGES, SWAP><<<grid, kThreads, C::kSmemBytes, st>>>(ma, mb, p);
+  gemm_nvfp4_kernel<BN, STAGES, SWAP><<<grid, C::kThreads, C::kSmemBytes, st>>>(ma, mb, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmArgs &g, int num_sms, cudaStream_t st) {
-  (void)num_sms;
-  if (g.M <= 32) return run<32, 6, true>(g, st);
-  return run<256, 4, false>(g, st);
+  if (g.M <= 32) return run<32, 6, true>(g, num_sms, st);
+  return run<256, 4, false>(g, num_sms, st);
 }
 
 }  // namespace nvfp4

@@ -81,6 +81,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// Whole-warp form of mbar_wait_bounded: every lane waits, then the warp reconverges and
+// agrees on the outcome, so warp-collective (.sync.aligned) instructions that follow run
+// with all 32 lanes together.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, uint64_t timeout_ns) {
+  const bool ok = mbar_wait_bounded(bar, parity, timeout_ns);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------------------ TMA
 
 // Untiled bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
@@ -261,6 +269,120 @@ __device__ __forceinline__ void unpack2(uint32_t w, float &lo, float &hi) {
     lo = f.x;
     hi = f.y;
   }
+}
+
+}  // namespace nvfp4
+
+namespace nvfp4 {
+
+// (a0, a1) * (b, b) with one packed fp32x2 multiply (two IEEE round-to-nearest products).
+__device__ __forceinline__ void mul2_rn(float a0, float a1, float b, float &d0, float &d1) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%1, %2};\n\t"
+      "mov.b64 rb, {%3, %3};\n\t"
+      "mul.rn.f32x2 %0, ra, rb;\n\t}"
+      : "=l"(d)
+      : "f"(a0), "f"(a1), "f"(b));
+  d0 = __uint_as_float(static_cast<uint32_t>(d));
+  d1 = __uint_as_float(static_cast<uint32_t>(d >> 32));
+}
+
+// Four E2M1 byte pairs -> one 32-bit word (byte j from pair j).
+__device__ __forceinline__ uint32_t e2m1x8_from_pairs(float y0, float y1, float y2, float y3,
+                                                     float y4, float y5, float y6, float y7) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
+  return out;
+}
+
+// max |x| over the 16 elements of 8 packed 16-bit words, in the input's own type (exact),
+// returned as fp32. max.xorsign.abs takes |a|, |b| for free; the sign it leaves (the xor of
+// the signs) is cleared at the end.
+template <int DTYPE>
+__device__ __forceinline__ float amax16_packed(const uint32_t (&w)[8]) {
+  uint32_t m0 = w[0], m1 = w[1];
+#pragma unroll
+  for (int i = 2; i < 8; i += 2) {
+    if constexpr (DTYPE == 0) {
+      asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m0) : "r"(w[i]));
+      asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m1) : "r"(w[i + 1]));
+    } else {
+      asm("max.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(m0) : "r"(w[i]));
+      asm("max.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(m1) : "r"(w[i + 1]));
+    }
+  }
+  if constexpr (DTYPE == 0) {
+    asm("max.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(m0) : "r"(m1));
+  } else {
+    asm("max.xorsign.abs.f16x2 %0, %0, %1;" : "+r"(m0) : "r"(m1));
+  }
+  const uint32_t m = m0 & 0x7FFF7FFFu;
+  float lo, hi;
+  if constexpr (DTYPE == 0) {
+    lo = __uint_as_float(m << 16);
+    hi = __uint_as_float(m & 0xFFFF0000u);
+  } else {
+    __half2 h = *reinterpret_cast<const __half2 *>(&m);
+    lo = __low2float(h);
+    hi = __high2float(h);
+  }
+  return fmaxf(lo, hi);
+}
+
+}  // namespace nvfp4
+
+namespace nvfp4 {
+
+// Packed fp32x2 arithmetic (sm_100a): two independent IEEE round-to-nearest results per
+// instruction, bit-identical to the scalar operations.
+struct F2 {
+  float x, y;
+};
+
+__device__ __forceinline__ F2 f2_from_u64(uint64_t v) {
+  return F2{__uint_as_float(static_cast<uint32_t>(v)), __uint_as_float(static_cast<uint32_t>(v >> 32))};
+}
+
+__device__ __forceinline__ F2 fma2_rn(F2 a, F2 b, F2 c) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%1, %2};\n\t"
+      "mov.b64 rb, {%3, %4};\n\t"
+      "mov.b64 rc, {%5, %6};\n\t"
+      "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return f2_from_u64(d);
+}
+
+__device__ __forceinline__ F2 mul2f_rn(F2 a, F2 b) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%1, %2};\n\t"
+      "mov.b64 rb, {%3, %4};\n\t"
+      "mul.rn.f32x2 %0, ra, rb;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return f2_from_u64(d);
+}
+
+__device__ __forceinline__ F2 add2f_rn(F2 a, F2 b) {
+  uint64_t d;
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%1, %2};\n\t"
+      "mov.b64 rb, {%3, %4};\n\t"
+      "add.rn.f32x2 %0, ra, rb;\n\t}"
+      : "=l"(d)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return f2_from_u64(d);
 }
 
 }  // namespace nvfp4

@@ -72,6 +72,64 @@ __device__ __forceinline__ uint64_t quant_block16(const float (&y)[16], float g,
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
+// E4M3 block scale of a block with maximum magnitude `amax` under encode scale g:
+// s = (amax / 6) * g (two IEEE roundings), saturating E4M3 code.
+__device__ __forceinline__ uint32_t block_scale_code(float amax, float g) {
+  return cvt_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), g));
+}
+
+// r = g / value(code) (IEEE division), 0 for a zero scale, clamped to FLT_MAX.
+__device__ __forceinline__ float block_recip(uint32_t code, float g) {
+  const float s_dec = e4m3_to_f32(code);
+  return (s_dec == 0.0f) ? 0.0f : fminf(__fdiv_rn(g, s_dec), FLT_MAX);
+}
+
+// Packs E2M1(x_i * r) for the 16 elements of 8 packed 16-bit words (element 2j in the low
+// nibble of byte j).
+template <int DTYPE>
+__device__ __forceinline__ uint64_t quant_packed16(const uint32_t (&w)[8], float r) {
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float lo, hi;
+    unpack2<DTYPE>(w[i], lo, hi);
+    mul2_rn(lo, hi, r, y[2 * i], y[2 * i + 1]);
+  }
+  const uint32_t a = e2m1x8_from_pairs(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+  const uint32_t b = e2m1x8_from_pairs(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+  return (static_cast<uint64_t>(b) << 32) | a;
+}
+
+// Same for 16 fp32 values.
+__device__ __forceinline__ uint64_t quant_f32x16(const float (&x)[16], float r) {
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mul2_rn(x[2 * i], x[2 * i + 1], r, y[2 * i], y[2 * i + 1]);
+  const uint32_t a = e2m1x8_from_pairs(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+  const uint32_t b = e2m1x8_from_pairs(y[8], y[9], y[10], y[11], y[12], y[13], y[14], y[15]);
+  return (static_cast<uint64_t>(b) << 32) | a;
+}
+
+// Per-CTA table of r for every finite E4M3 scale code under one encode scale g
+// (128 entries; entry 0x7F is never indexed: codes come from a saturating conversion).
+__device__ __forceinline__ void fill_recip_table(float *table, float g) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) table[c] = (c == 0x7F) ? 0.0f : block_recip(c, g);
+}
+
+// Byte offset of row r's scale for column c = 0 (the per-row part of sf_offset).
+__device__ __forceinline__ int64_t sf_row_base(int layout, int64_t r, int64_t C, int64_t Cp) {
+  if (layout == kSf128x4) return ((r >> 7) * (Cp >> 2) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2);
+  if (layout == kSf8x4) return ((r >> 3) * (Cp >> 2) << 5) + ((r & 7) << 2);
+  return r * C;
+}
+
+// Column part of sf_offset (add to sf_row_base).
+__device__ __forceinline__ int64_t sf_col_off(int layout, int64_t c) {
+  if (layout == kSf128x4) return ((c >> 2) << 9) + (c & 3);
+  if (layout == kSf8x4) return ((c >> 2) << 5) + (c & 3);
+  return c;
+}
+
 template <int DTYPE>
 __device__ __forceinline__ void unpack16(const uint32_t (&w)[8], float (&y)[16]) {
 #pragma unroll
@@ -151,39 +209,43 @@ __global__ void __launch_bounds__(1024) amax_finalize_kernel(const float *__rest
 
 // ------------------------------------------------------------------------------ streaming
 
-// One thread per 16-element block, UNROLL blocks in flight per thread.
-// g_per_row == 0: g[0] for every row; == 1: g[r].
+// Row-major streaming quantize: CTA b handles rows b, b + gridDim.x, ...; thread t owns
+// blocks t, t + blockDim.x, ... of each row (one 32-byte block per load), UNROLL blocks in
+// flight per thread. g_per_row == 0: g[0] for every row (r from a per-CTA table of all E4M3
+// codes); == 1: g[r] (r by division).
 template <int DTYPE, int UNROLL, bool V8>
 __global__ void __launch_bounds__(256) quant_stream_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, const float *__restrict__ g,
     int g_per_row, uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp,
     int64_t Cp) {
-  const int64_t C = K / 16;
-  const int64_t nblk = M * C;
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  __shared__ float rtab[128];
+  const int C = static_cast<int>(K / 16);
   const float g0 = g_per_row ? 0.0f : g[0];
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < nblk;
-       base += nthreads * UNROLL) {
-    uint32_t w[UNROLL][8];
+  if (!g_per_row) fill_recip_table(rtab, g0);
+  __syncthreads();
+  const int step = blockDim.x * UNROLL;
+  for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
+    const uint16_t *xrow = x + r * ldx;
+    uint8_t *qrow = q + r * (K / 2);
+    uint8_t *sfrow = sf + sf_row_base(layout, r, C, Cp);
+    const float gr = g_per_row ? g[r] : g0;
+    for (int c0 = threadIdx.x; c0 < C; c0 += step) {
+      uint32_t w[UNROLL][8];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int64_t b = base + u * nthreads;
-      if (b < nblk) {
-        const int64_t r = b / C, c = b - r * C;
-        ld_block16<V8>(x + r * ldx + c * 16, w[u]);
+      for (int u = 0; u < UNROLL; ++u) {
+        const int c = c0 + u * blockDim.x;
+        if (c < C) ld_block16<V8>(xrow + c * 16, w[u]);
       }
-    }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int64_t b = base + u * nthreads;
-      if (b < nblk) {
-        const int64_t r = b / C, c = b - r * C;
-        float y[16];
-        unpack16<DTYPE>(w[u], y);
-        uint32_t s;
-        const uint64_t packed = quant_block16(y, g_per_row ? g[r] : g0, s);
-        st_cs_u64(q + r * (K / 2) + c * 8, packed);
-        sf[sf_offset(layout, r, c, C, Cp)] = static_cast<uint8_t>(s);
+      for (int u = 0; u < UNROLL; ++u) {
+        const int c = c0 + u * blockDim.x;
+        if (c < C) {
+          const float amax = amax16_packed<DTYPE>(w[u]);
+          const uint32_t s = block_scale_code(amax, gr);
+          const float rr = g_per_row ? block_recip(s, gr) : rtab[s];
+          st_cs_u64(qrow + c * 8, quant_packed16<DTYPE>(w[u], rr));
+          sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);
+        }
       }
     }
   }
@@ -214,19 +276,25 @@ __global__ void __launch_bounds__(256) row_scale_kernel(const uint16_t *__restri
 
 // ------------------------------------------------------------------------------ per-token
 
-// Persistent: CTA b handles rows b, b + gridDim.x, ... Each row (K * 2 bytes) is brought into
-// one of `stages` shared-memory slots by a bulk TMA copy issued by thread 0 `stages` rows
-// ahead; all threads then reduce the row amax and quantize the row from shared memory.
-template <int DTYPE>
+// Persistent: CTA b handles rows b, b + gridDim.x, ... Each row (K * 2 bytes) is brought
+// into one of `stages` shared-memory slots by a bulk TMA copy that thread 0 issues `stages`
+// rows ahead. Thread t owns blocks t, t + nthreads, ... (at most BPT): it reads them from
+// shared memory once, keeps them in registers with their block maxima, joins one CTA
+// barrier for the row maximum (the barrier also carries the bounded-wait vote, and after it
+// the slot is refilled), then quantizes its blocks from registers.
+template <int DTYPE, int BPT>
 __global__ void __launch_bounds__(256) quant_pertoken_rowcache_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float *__restrict__ g,
     uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp, int64_t Cp,
     int stages) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ uint64_t full[kRowcacheMaxStages];
-  __shared__ float red[32];
-  const int64_t C = K / 16;
+  __shared__ float red[2][8];
+  const int C = static_cast<int>(K / 16);
   const uint32_t row_bytes = static_cast<uint32_t>(K * 2);
+  const int nthreads = blockDim.x;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = nthreads >> 5;
 
   zero_sf_padding(sf, layout, M, C, Rp, Cp);
 
@@ -247,51 +315,38 @@ __global__ void __launch_bounds__(256) quant_pertoken_rowcache_kernel(
       }
     }
   }
-
-  int64_t j = 0;
+  int stage = 0;
+  uint32_t parity = 0;
+  uint32_t j = 0;
   for (int64_t r = first; r < M; r += step, ++j) {
-    const int stage = static_cast<int>(j % stages);
-    const uint32_t parity = static_cast<uint32_t>((j / stages) & 1);
-    // Bounded wait; every thread takes the same decision so the CTA leaves together.
     const bool ok = mbar_wait_bounded(&full[stage], parity, kWaitTimeoutNs);
+    const uint8_t *row = smem + static_cast<size_t>(stage) * row_bytes;
+
+    uint32_t w[BPT][8];
+    float bam[BPT];
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      const int c = threadIdx.x + i * nthreads;
+      bam[i] = 0.0f;
+      if (c < C) {
+        const uint4 *p = reinterpret_cast<const uint4 *>(row + c * 32);
+        const uint4 a = p[0], b = p[1];
+        w[i][0] = a.x; w[i][1] = a.y; w[i][2] = a.z; w[i][3] = a.w;
+        w[i][4] = b.x; w[i][5] = b.y; w[i][6] = b.z; w[i][7] = b.w;
+        bam[i] = amax16_packed<DTYPE>(w[i]);
+        m = fmaxf(m, bam[i]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane_id() == 0) red[j & 1][warp] = m;
+    // One barrier per row: row-maximum partials are visible, every thread is done reading the
+    // slot, and a timed-out wait anywhere makes the whole CTA leave together.
     if (__syncthreads_or(!ok)) {
       if (threadIdx.x == 0) atomicOr(&g_device_error, kDevErrTimeout);
       return;
     }
-    const uint8_t *row = smem + static_cast<size_t>(stage) * row_bytes;
-
-    // Row amax: plain 16-byte chunks in order (conflict-free).
-    float m = 0.0f;
-    const uint4 *chunks = reinterpret_cast<const uint4 *>(row);
-    for (int64_t i = threadIdx.x; i < static_cast<int64_t>(row_bytes / 16); i += blockDim.x) {
-      const uint4 a = chunks[i];
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float lo, hi;
-        unpack2<DTYPE>(w[k], lo, hi);
-        m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
-      }
-    }
-    const float gr = global_scale_from_amax(block_max(m, red));
-    if (threadIdx.x == 0) g[r] = gr;
-
-    // Each thread quantizes whole 32-byte blocks; lanes 4-7 of each quarter-warp read the
-    // upper half first so the 8 lanes of a 128-bit shared-memory phase hit distinct banks.
-    const uint32_t h = (threadIdx.x >> 2) & 1u;
-    for (int64_t c = threadIdx.x; c < C; c += blockDim.x) {
-      const uint4 *p = reinterpret_cast<const uint4 *>(row + c * 32);
-      const uint4 first = p[h], second = p[h ^ 1u];
-      const uint4 a = h ? second : first, b = h ? first : second;
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-      float y[16];
-      unpack16<DTYPE>(w, y);
-      uint32_t s;
-      const uint64_t packed = quant_block16(y, gr, s);
-      st_cs_u64(q + r * (K / 2) + c * 8, packed);
-      sf[sf_offset(layout, r, c, C, Cp)] = static_cast<uint8_t>(s);
-    }
-    __syncthreads();  // every thread is done with this slot
     if (threadIdx.x == 0) {
       const int64_t rn = r + static_cast<int64_t>(stages) * step;
       if (rn < M) {
@@ -300,71 +355,119 @@ __global__ void __launch_bounds__(256) quant_pertoken_rowcache_kernel(
                  &full[stage]);
       }
     }
+    float amax = red[j & 1][0];
+    for (int w2 = 1; w2 < nwarps; ++w2) amax = fmaxf(amax, red[j & 1][w2]);
+    const float gr = global_scale_from_amax(amax);
+    if (threadIdx.x == 0) g[r] = gr;
+
+    uint8_t *qrow = q + r * (K / 2);
+    uint8_t *sfrow = sf + sf_row_base(layout, r, C, Cp);
+#pragma unroll
+    for (int i = 0; i < BPT; ++i) {
+      const int c = threadIdx.x + i * nthreads;
+      if (c < C) {
+        const uint32_t s = block_scale_code(bam[i], gr);
+        const float rr = block_recip(s, gr);
+        st_cs_u64(qrow + c * 8, quant_packed16<DTYPE>(w[i], rr));
+        sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);
+      }
+    }
+    if (++stage == stages) {
+      stage = 0;
+      parity ^= 1u;
+    }
   }
 }
 
 // ------------------------------------------------------------------------------ SwiGLU
 
-// Library fp32 exponential: clamp to [-87, 88]; k = rint(v * log2 e); Cody-Waite reduction
-// f = v - k*ln2_hi - k*ln2_lo; degree-7 Taylor polynomial of e^f (coefficients 1/n!
-// rounded to fp32) by fused multiply-add; times 2^k built from exponent bits.
-__device__ __forceinline__ float exp_f32(float v) {
-  v = fminf(fmaxf(v, -87.0f), 88.0f);
-  const float k = rintf(__fmul_rn(v, 0x1.715476p+0f));
-  float f = __fmaf_rn(-k, 0x1.62e4p-1f, v);
-  f = __fmaf_rn(-k, 0x1.7f7d1cp-20f, f);
-  float p = 0x1.a01a02p-13f;             // 1/7!
-  p = __fmaf_rn(p, f, 0x1.6c16c2p-10f);  // 1/6!
-  p = __fmaf_rn(p, f, 0x1.111112p-7f);   // 1/5!
-  p = __fmaf_rn(p, f, 0x1.555556p-5f);   // 1/4!
-  p = __fmaf_rn(p, f, 0x1.555556p-3f);   // 1/3!
-  p = __fmaf_rn(p, f, 0.5f);             // 1/2!
-  p = __fmaf_rn(p, f, 1.0f);             // 1/1!
-  p = __fmaf_rn(p, f, 1.0f);             // 1/0!
-  const float two_k = __int_as_float((static_cast<int>(k) + 127) << 23);
-  return __fmul_rn(p, two_k);
+// Library fp32 exponential on a pair of values: clamp to [-87, 88]; k = rint(v * log2 e);
+// Cody-Waite reduction f = v - k*ln2_hi - k*ln2_lo; degree-7 Taylor polynomial of e^f
+// (coefficients 1/n! rounded to fp32) by fused multiply-add; times 2^k built from exponent
+// bits. Packed fp32x2 instructions give each lane the same IEEE results as scalar code.
+// rint is taken as (z + 1.5*2^23) - 1.5*2^23: for |z| < 2^22 the sum is rounded to an
+// integer with ties to even, which is exactly rint(z), and its low mantissa bits are k.
+__device__ __forceinline__ F2 exp2_f32(F2 v) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  v.x = fminf(fmaxf(v.x, -87.0f), 88.0f);
+  v.y = fminf(fmaxf(v.y, -87.0f), 88.0f);
+  const F2 z = mul2f_rn(v, F2{0x1.715476p+0f, 0x1.715476p+0f});
+  const F2 t = add2f_rn(z, F2{kRound, kRound});
+  const F2 k = add2f_rn(t, F2{-kRound, -kRound});
+  const F2 nk{-k.x, -k.y};
+  F2 f = fma2_rn(nk, F2{0x1.62e4p-1f, 0x1.62e4p-1f}, v);
+  f = fma2_rn(nk, F2{0x1.7f7d1cp-20f, 0x1.7f7d1cp-20f}, f);
+  F2 p{0x1.a01a02p-13f, 0x1.a01a02p-13f};                   // 1/7!
+  p = fma2_rn(p, f, F2{0x1.6c16c2p-10f, 0x1.6c16c2p-10f});  // 1/6!
+  p = fma2_rn(p, f, F2{0x1.111112p-7f, 0x1.111112p-7f});    // 1/5!
+  p = fma2_rn(p, f, F2{0x1.555556p-5f, 0x1.555556p-5f});    // 1/4!
+  p = fma2_rn(p, f, F2{0x1.555556p-3f, 0x1.555556p-3f});    // 1/3!
+  p = fma2_rn(p, f, F2{0.5f, 0.5f});                        // 1/2!
+  p = fma2_rn(p, f, F2{1.0f, 1.0f});                        // 1/1!
+  p = fma2_rn(p, f, F2{1.0f, 1.0f});                        // 1/0!
+  // 2^k: k sits in the low bits of t (t's bits = 0x4B400000 + k), so (k + 127) << 23 is
+  // (bits(t) - 0x4B400000 + 127) << 23.
+  const F2 two_k{__int_as_float((__float_as_int(t.x) - 0x4B3FFF81) << 23),
+                 __int_as_float((__float_as_int(t.y) - 0x4B3FFF81) << 23)};
+  return mul2f_rn(p, two_k);
 }
 
-__device__ __forceinline__ float swiglu_f32(float gate, float up) {
-  const float silu = __fdiv_rn(gate, __fadd_rn(1.0f, exp_f32(-gate)));
-  return __fmul_rn(silu, up);
+// y = silu(gate) * up = gate / (1 + e(-gate)) * up for a pair of elements.
+__device__ __forceinline__ F2 swiglu2_f32(F2 gate, F2 up) {
+  const F2 e = exp2_f32(F2{-gate.x, -gate.y});
+  const F2 den = add2f_rn(F2{1.0f, 1.0f}, e);
+  const F2 silu{__fdiv_rn(gate.x, den.x), __fdiv_rn(gate.y, den.y)};
+  return mul2f_rn(silu, up);
 }
 
+// Row-major like quant_stream_kernel: CTA b handles rows b, b + gridDim.x, ...; thread t
+// owns blocks t, t + blockDim.x, ... of the output row (gate and up loaded as two 32-byte
+// blocks each).
 template <int DTYPE, int UNROLL, bool V8>
 __global__ void __launch_bounds__(256) swiglu_quant_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t H, int64_t ldx, const float *__restrict__ g,
     uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp, int64_t Cp) {
-  const int64_t C = H / 16;
-  const int64_t nblk = M * C;
-  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  __shared__ float rtab[128];
+  const int C = static_cast<int>(H / 16);
   const float g0 = g[0];
-  for (int64_t base = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; base < nblk;
-       base += nthreads * UNROLL) {
-    uint32_t wg[UNROLL][8], wu[UNROLL][8];
+  fill_recip_table(rtab, g0);
+  __syncthreads();
+  const int step = blockDim.x * UNROLL;
+  for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
+    const uint16_t *grow = x + r * ldx;
+    const uint16_t *urow = grow + H;
+    uint8_t *qrow = q + r * (H / 2);
+    uint8_t *sfrow = sf + sf_row_base(layout, r, C, Cp);
+    for (int c0 = threadIdx.x; c0 < C; c0 += step) {
+      uint32_t wg[UNROLL][8], wu[UNROLL][8];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int64_t b = base + u * nthreads;
-      if (b < nblk) {
-        const int64_t r = b / C, c = b - r * C;
-        const uint16_t *row = x + r * ldx;
-        ld_block16<V8>(row + c * 16, wg[u]);
-        ld_block16<V8>(row + H + c * 16, wu[u]);
+      for (int u = 0; u < UNROLL; ++u) {
+        const int c = c0 + u * blockDim.x;
+        if (c < C) {
+          ld_block16<V8>(grow + c * 16, wg[u]);
+          ld_block16<V8>(urow + c * 16, wu[u]);
+        }
       }
-    }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int64_t b = base + u * nthreads;
-      if (b < nblk) {
-        const int64_t r = b / C, c = b - r * C;
-        float gate[16], up[16], y[16];
-        unpack16<DTYPE>(wg[u], gate);
-        unpack16<DTYPE>(wu[u], up);
+      for (int u = 0; u < UNROLL; ++u) {
+        const int c = c0 + u * blockDim.x;
+        if (c < C) {
+          float y[16];
+          float amax = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = swiglu_f32(gate[i], up[i]);
-        uint32_t s;
-        const uint64_t packed = quant_block16(y, g0, s);
-        st_cs_u64(q + r * (H / 2) + c * 8, packed);
-        sf[sf_offset(layout, r, c, C, Cp)] = static_cast<uint8_t>(s);
+          for (int i = 0; i < 8; ++i) {
+            F2 gate, up;
+            unpack2<DTYPE>(wg[u][i], gate.x, gate.y);
+            unpack2<DTYPE>(wu[u][i], up.x, up.y);
+            const F2 v = swiglu2_f32(gate, up);
+            y[2 * i] = v.x;
+            y[2 * i + 1] = v.y;
+            amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+          }
+          const uint32_t s = block_scale_code(amax, g0);
+          st_cs_u64(qrow + c * 8, quant_f32x16(y, rtab[s]));
+          sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);
+        }
       }
     }
   }
@@ -394,6 +497,27 @@ __global__ void sf_unswizzle_kernel(const uint8_t *__restrict__ in, uint8_t *__r
 }
 
 // ------------------------------------------------------------------------------ launchers
+
+// Threads per CTA for a row of C blocks handled UNROLL at a time: a multiple of 32, at most
+// 256, so that the row splits into whole rounds of threads x UNROLL as evenly as possible.
+static int row_threads(int64_t C, int unroll) {
+  const int64_t per_round = (C + unroll - 1) / unroll;
+  const int64_t rounds = (per_round + 255) / 256;
+  int64_t t = (per_round + rounds - 1) / rounds;
+  t = (t + 31) / 32 * 32;
+  if (t < 32) t = 32;
+  if (t > 256) t = 256;
+  return static_cast<int>(t);
+}
+
+static int row_grid(int64_t M, int threads, int num_sms) {
+  int64_t per_sm = 2048 / threads;
+  if (per_sm > 16) per_sm = 16;
+  int64_t g = static_cast<int64_t>(num_sms) * per_sm;
+  if (g > M) g = M;
+  if (g < 1) g = 1;
+  return static_cast<int>(g);
+}
 
 static int grid_for(int64_t work_items, int threads, int max_ctas) {
   int64_t g = (work_items + threads - 1) / threads;
@@ -451,56 +575,73 @@ cudaError_t launch_quantize(const void *x, int dtype, int64_t M, int64_t K, int6
                             int per_token, uint8_t *q, uint8_t *sf, int layout, int64_t Rp,
                             int64_t Cp, int num_sms, int max_smem_optin, cudaStream_t st) {
   const uint16_t *xp = static_cast<const uint16_t *>(x);
-  const int64_t nblk = M * (K / 16);
   const bool v8 = blocks_32b_aligned(x, ldx);
   if (!per_token) {
-    const int grid = grid_for(nblk, 256, num_sms * 8);
+    const int threads = row_threads(K / 16, 2);
+    const int grid = row_grid(M, threads, num_sms);
     NVFP4_DISPATCH_DT_V8(dtype, v8,
-                         (quant_stream_kernel<DT, 2, VV><<<grid, 256, 0, st>>>(
+                         (quant_stream_kernel<DT, 2, VV><<<grid, threads, 0, st>>>(
                              xp, M, K, ldx, g, 0, q, sf, layout, Rp, Cp)));
     return cudaGetLastError();
   }
   const int64_t row_bytes = K * 2;
-  // Rows in flight per CTA: up to kRowcacheMaxStages, fewer when three CTAs of that size would
-  // not share an SM; at least two or the row is not staged at all.
-  int stages = 0;
-  for (int s = kRowcacheMaxStages; s >= 2; --s) {
-    if (row_bytes * s + 1024 <= max_smem_optin) {
-      stages = s;
-      break;
+  const int C = static_cast<int>(K / 16);
+  // Blocks per thread: the smallest power of two that keeps a row within 256 threads.
+  int bpt = 1;
+  while (bpt <= 8 && (static_cast<int64_t>(C) + bpt - 1) / bpt > 256) bpt *= 2;
+  int stages = 0, per_sm = 0;
+  int nthreads = 0;
+  if (bpt <= 8) {
+    nthreads = static_cast<int>(((C + bpt - 1) / bpt + 31) / 32 * 32);
+    // Rows in flight per SM = CTAs per SM x stages, within ~220 KB of shared memory and
+    // 2048 threads per SM; prefer more CTAs on a tie.
+    for (int s = 2; s <= 4 && s <= kRowcacheMaxStages; ++s) {
+      const int64_t smem = row_bytes * s + 1024;
+      if (smem > max_smem_optin) break;
+      int cps = static_cast<int>((220 * 1024) / smem);
+      if (cps > 2048 / nthreads) cps = 2048 / nthreads;
+      if (cps > 32) cps = 32;
+      if (cps >= 1 && cps * s > per_sm * stages) {
+        stages = s;
+        per_sm = cps;
+      }
     }
   }
   if (stages >= 2) {
-    while (stages > 2 && row_bytes * stages * 3 > 220 * 1024) --stages;
     const size_t smem = static_cast<size_t>(row_bytes * stages);
-    int per_sm = static_cast<int>((220 * 1024) / (smem + 2048));
-    if (per_sm < 1) per_sm = 1;
-    if (per_sm > 8) per_sm = 8;
     int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
     if (grid > M) grid = M;
     if (grid < 1) grid = 1;
-    cudaError_t e;
+#define NVFP4_LAUNCH_ROWCACHE(DT, B)                                                          \
+  do {                                                                                        \
+    cudaError_t e = cudaFuncSetAttribute(quant_pertoken_rowcache_kernel<DT, B>,               \
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,         \
+                                         static_cast<int>(smem));                             \
+    if (e != cudaSuccess) return e;                                                           \
+    quant_pertoken_rowcache_kernel<DT, B><<<static_cast<int>(grid), nthreads, smem, st>>>(   \
+        xp, M, K, ldx, g, q, sf, layout, Rp, Cp, stages);                                     \
+  } while (0)
     if (dtype == kInBf16) {
-      e = cudaFuncSetAttribute(quant_pertoken_rowcache_kernel<0>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      quant_pertoken_rowcache_kernel<0><<<static_cast<int>(grid), 256, smem, st>>>(
-          xp, M, K, ldx, g, q, sf, layout, Rp, Cp, stages);
+      if (bpt == 1) NVFP4_LAUNCH_ROWCACHE(0, 1);
+      else if (bpt == 2) NVFP4_LAUNCH_ROWCACHE(0, 2);
+      else if (bpt == 4) NVFP4_LAUNCH_ROWCACHE(0, 4);
+      else NVFP4_LAUNCH_ROWCACHE(0, 8);
     } else {
-      e = cudaFuncSetAttribute(quant_pertoken_rowcache_kernel<1>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      quant_pertoken_rowcache_kernel<1><<<static_cast<int>(grid), 256, smem, st>>>(
-          xp, M, K, ldx, g, q, sf, layout, Rp, Cp, stages);
+      if (bpt == 1) NVFP4_LAUNCH_ROWCACHE(1, 1);
+      else if (bpt == 2) NVFP4_LAUNCH_ROWCACHE(1, 2);
+      else if (bpt == 4) NVFP4_LAUNCH_ROWCACHE(1, 4);
+      else NVFP4_LAUNCH_ROWCACHE(1, 8);
     }
+#undef NVFP4_LAUNCH_ROWCACHE
     return cudaGetLastError();
   }
   // Rows too long to stage: row amax pass, then the streaming pass with per-row g.
   const int rgrid = static_cast<int>(M < num_sms * 8 ? M : num_sms * 8);
-  const int grid = grid_for(nblk, 256, num_sms * 8);
+  const int threads = row_threads(K / 16, 2);
+  const int grid = row_grid(M, threads, num_sms);
   NVFP4_DISPATCH_DT_V8(dtype, v8, (row_scale_kernel<DT, VV><<<rgrid, 256, 0, st>>>(xp, M, K, ldx, g)));
   NVFP4_DISPATCH_DT_V8(dtype, v8,
-                       (quant_stream_kernel<DT, 2, VV><<<grid, 256, 0, st>>>(
+                       (quant_stream_kernel<DT, 2, VV><<<grid, threads, 0, st>>>(
                            xp, M, K, ldx, g, 1, q, sf, layout, Rp, Cp)));
   return cudaGetLastError();
 }
@@ -509,11 +650,11 @@ cudaError_t launch_swiglu_quantize(const void *x, int dtype, int64_t M, int64_t 
                                    const float *g, uint8_t *q, uint8_t *sf, int layout, int64_t Rp,
                                    int64_t Cp, int num_sms, cudaStream_t st) {
   const uint16_t *xp = static_cast<const uint16_t *>(x);
-  const int64_t nblk = M * (H / 16);
-  const int grid = grid_for(nblk, 256, num_sms * 8);
+  const int threads = row_threads(H / 16, 2);
+  const int grid = row_grid(M, threads, num_sms);
   const bool v8 = blocks_32b_aligned(x, ldx);
   NVFP4_DISPATCH_DT_V8(dtype, v8,
-                       (swiglu_quant_kernel<DT, 2, VV><<<grid, 256, 0, st>>>(
+                       (swiglu_quant_kernel<DT, 2, VV><<<grid, threads, 0, st>>>(
                            xp, M, H, ldx, g, q, sf, layout, Rp, Cp)));
   return cudaGetLastError();
 }
