@@ -16,13 +16,10 @@ replicas (weak scaling): the path has no exchange step.
 from __future__ import annotations
 
 import argparse
-import csv
 import hashlib
-import io
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -69,50 +66,89 @@ def algorithmic(workload, M=None, K=None, N=None, H=None, a_layout="128x4"):
 
 
 class Clocks:
-    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
+    """Samples the SM clock and the clock-event (throttle) reasons while the timed region runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    A thread polls NVML back to back (a query takes well under a millisecond), so even a
+    timed region of a few milliseconds gets samples. One sample is also taken right before
+    and right after the region; if the region was too short for the thread to land a sample
+    inside it, those two bracketing samples are reported and `window` says so. Falls back
+    to `nvidia-smi -lms 100` when NVML cannot be loaded."""
+
+    REASONS = {  # NVML clocks-event reason bits
+        "hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
 
     def __init__(self, bus_id=None):
         self.bus_id = bus_id
-        self.proc = None
+        self.inside, self.bracket = [], []
+        self.max_mhz = None
+        self.nv = None
+        self.handle = None
+        self.thread = None
+        self.stop = False
+
+    def _sample(self):
+        nv = self.nv
+        try:
+            mhz = nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM)
+            fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            return (float(mhz), int(fn(self.handle)))
+        except Exception:
+            return None
+
+    def _poll(self):
+        while not self.stop:
+            s = self._sample()
+            if s is not None:
+                self.inside.append(s)
+            time.sleep(0.0002)
 
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-               "-lms", "100"]
-        if self.bus_id:
-            cmd += ["-i", self.bus_id]
+        if self.bus_id is None:
+            return self
         try:
-            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+
+            nv.nvmlInit()
+            self.nv = nv
+            self.handle = nv.nvmlDeviceGetHandleByPciBusId(self.bus_id)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.handle, nv.NVML_CLOCK_SM))
+        except Exception:
+            self.nv = None
+            return self
+        s = self._sample()
+        if s is not None:
+            self.bracket.append(s)
+        import threading
+
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
+        if self.thread is not None:
+            self.stop = True
+            self.thread.join()
+            s = self._sample()
+            if s is not None:
+                self.bracket.append(s)
+        if self.nv is not None:
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                self.nv.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self):
-        rows = [r for r in csv.reader(io.StringIO(self.out or "")) if len(r) >= 9]
+        rows, window = self.inside, "inside"
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]
-                          and "Not" not in r[5 + i]})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+            rows, window = self.bracket, "bracketing"
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"]}
+        reasons = sorted({name for _, bits in rows for name, b in self.REASONS.items() if bits & b})
+        return {"sm_mhz": statistics.median(m for m, _ in rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows), "window": window, "source": "nvml"}
 
 
 def _source_hash(*rel):
@@ -467,8 +503,8 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="per_token",
                     choices=["per_token", "swiglu", "decode", "prefill", "tiny"])

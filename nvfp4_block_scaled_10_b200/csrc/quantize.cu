@@ -72,10 +72,46 @@ __device__ __forceinline__ uint64_t quant_block16(const float (&y)[16], float g,
   return (static_cast<uint64_t>(hi) << 32) | lo;
 }
 
+// fl(x / 6) for x >= 0 (a block maximum), the IEEE quotient, without the general division
+// sequence: q0 = fl(x * fl(1/6)), rem = x - 6*q0 by one FMA, q1 = q0 + rem*fl(1/6) by one
+// FMA. An exhaustive check over every fp32 bit pattern with a clear sign bit finds q1
+// equal to the IEEE quotient for +0 and every finite x >= 2^-125 (NaN and infinity keep
+// q0, which is then the quotient too); for 0 < x < 2^-125 the quotient is subnormal and the
+// IEEE division is used.
+__device__ __forceinline__ float div6_rn(float x) {
+  if (x > 0.0f && x < 0x1p-125f) return __fdiv_rn(x, 6.0f);
+  constexpr float kSixth = 0x1.555556p-3f;  // fl(1/6)
+  const float q0 = __fmul_rn(x, kSixth);
+  const float rem = __fmaf_rn(-q0, 6.0f, x);
+  const float q1 = __fmaf_rn(rem, kSixth, q0);
+  return (rem == rem) ? q1 : q0;
+}
+
 // E4M3 block scale of a block with maximum magnitude `amax` under encode scale g:
 // s = (amax / 6) * g (two IEEE roundings), saturating E4M3 code.
 __device__ __forceinline__ uint32_t block_scale_code(float amax, float g) {
-  return cvt_e4m3(__fmul_rn(__fdiv_rn(amax, 6.0f), g));
+  return cvt_e4m3(__fmul_rn(div6_rn(amax), g));
+}
+
+// Per-row reciprocal table for one warp: lane k (1..15) holds fl(g / k), lane 0 holds 0.
+// Every finite E4M3 value is k * 2^E with an integer k in 0..15 (k = 8 + mantissa for a
+// normal code with E = exponent - 10, k = mantissa with E = -9 for a subnormal code), so
+// g / value = fl(g / k) * 2^-E exactly whenever the product is a normal float, and an
+// overflow of the product is exactly an overflow of the quotient. For every g that
+// global_scale_from_amax yields from a bf16 or fp16 maximum the products are normal; an
+// exhaustive check over those g and all 127 codes finds the table equal to the division.
+__device__ __forceinline__ float row_recip_lane(float g) {
+  const int k = static_cast<int>(lane_id());
+  return (k == 0 || k > 15) ? 0.0f : __fdiv_rn(g, static_cast<float>(k));
+}
+
+// r = g / value(code) from the warp's row table (all 32 lanes must call it together).
+__device__ __forceinline__ float row_recip(uint32_t code, float lane_tab) {
+  const uint32_t e = code >> 3, m = code & 7u;
+  const int k = static_cast<int>(e ? (8u | m) : m);
+  const float t = __shfl_sync(0xffffffffu, lane_tab, k);
+  const float p2 = __uint_as_float((137u - (e ? e : 1u)) << 23);  // 2^(10 - max(e, 1))
+  return fminf(__fmul_rn(t, p2), FLT_MAX);
 }
 
 // r = g / value(code) (IEEE division), 0 for a zero scale, clamped to FLT_MAX.
@@ -359,15 +395,17 @@ __global__ void __launch_bounds__(256) quant_pertoken_rowcache_kernel(
     for (int w2 = 1; w2 < nwarps; ++w2) amax = fmaxf(amax, red[j & 1][w2]);
     const float gr = global_scale_from_amax(amax);
     if (threadIdx.x == 0) g[r] = gr;
+    const float tab = row_recip_lane(gr);
 
     uint8_t *qrow = q + r * (K / 2);
     uint8_t *sfrow = sf + sf_row_base(layout, r, C, Cp);
 #pragma unroll
     for (int i = 0; i < BPT; ++i) {
       const int c = threadIdx.x + i * nthreads;
+      // out-of-row slots carry bam = 0 (code 0) and still join the table shuffle
+      const uint32_t s = block_scale_code(bam[i], gr);
+      const float rr = row_recip(s, tab);
       if (c < C) {
-        const uint32_t s = block_scale_code(bam[i], gr);
-        const float rr = block_recip(s, gr);
         st_cs_u64(qrow + c * 8, quant_packed16<DTYPE>(w[i], rr));
         sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);
       }
@@ -586,9 +624,13 @@ cudaError_t launch_quantize(const void *x, int dtype, int64_t M, int64_t K, int6
   }
   const int64_t row_bytes = K * 2;
   const int C = static_cast<int>(K / 16);
-  // Blocks per thread: the smallest power of two that keeps a row within 256 threads.
+  // Blocks per thread: the smallest power of two that keeps a row within 128 threads
+  // (within 256 once 8 blocks per thread no longer suffice). Four blocks per thread on a
+  // 128-thread CTA was the fastest shape measured for 7168-wide rows: fewer CTA barriers
+  // per row than 2 x 224 threads, more rows in flight than one warp per row.
   int bpt = 1;
-  while (bpt <= 8 && (static_cast<int64_t>(C) + bpt - 1) / bpt > 256) bpt *= 2;
+  while (bpt < 8 && (static_cast<int64_t>(C) + bpt - 1) / bpt > 128) bpt *= 2;
+  if ((static_cast<int64_t>(C) + bpt - 1) / bpt > 256) bpt = 16;
   int stages = 0, per_sm = 0;
   int nthreads = 0;
   if (bpt <= 8) {
