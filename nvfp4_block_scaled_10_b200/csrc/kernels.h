@@ -13,7 +13,6 @@ constexpr int kSf8x4 = 2;
 constexpr int kInBf16 = 0;
 constexpr int kInFp16 = 1;
 
-constexpr int kRowcacheMaxStages = 6;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s without progress
 constexpr int kDevErrTimeout = 1;
 

@@ -81,6 +81,32 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
+// try_wait with an explicit suspend-time hint: a thread whose phase is not complete sleeps
+// until the phase completes or about `hint_ns` pass, instead of retrying after the short
+// system-dependent default; waiting warps then take no issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait built on the sleeping try_wait; gives up (returns false) after timeout_ns.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+                                                uint32_t hint_ns) {
+  if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+    if (globaltimer_ns() - t0 > timeout_ns) return false;
+  }
+}
+
 // Whole-warp form of mbar_wait_bounded: every lane waits, then the warp reconverges and
 // agrees on the outcome, so warp-collective (.sync.aligned) instructions that follow run
 // with all 32 lanes together.

@@ -312,107 +312,84 @@ __global__ void __launch_bounds__(256) row_scale_kernel(const uint16_t *__restri
 
 // ------------------------------------------------------------------------------ per-token
 
-// Persistent: CTA b handles rows b, b + gridDim.x, ... Each row (K * 2 bytes) is brought
-// into one of `stages` shared-memory slots by a bulk TMA copy that thread 0 issues `stages`
-// rows ahead. Thread t owns blocks t, t + nthreads, ... (at most BPT): it reads them from
-// shared memory once, keeps them in registers with their block maxima, joins one CTA
-// barrier for the row maximum (the barrier also carries the bounded-wait vote, and after it
-// the slot is refilled), then quantizes its blocks from registers.
+// Persistent, one row per CTA at a time: CTA b handles rows b, b + gridDim.x, ... Thread t
+// owns blocks t + i * NT (i < BPT) of a row and holds them in registers, so the row is read
+// from HBM once: block maxima from registers, one CTA barrier for the row maximum, then the
+// blocks are quantized from the same registers. As soon as block i of the current row has
+// been quantized, block i of the CTA's next row is loaded into the registers it occupied,
+// so the next row streams in while the rest of this one is being quantized. (Staging the
+// rows in shared memory by bulk copies with a deeper ring measured slower than this on
+// 8192 x 7168 bf16 rows.)
 template <int DTYPE, int BPT>
-__global__ void __launch_bounds__(256) quant_pertoken_rowcache_kernel(
-    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float *__restrict__ g,
-    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp, int64_t Cp,
-    int stages) {
-  extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ uint64_t full[kRowcacheMaxStages];
-  __shared__ float red[2][8];
-  const int C = static_cast<int>(K / 16);
-  const uint32_t row_bytes = static_cast<uint32_t>(K * 2);
-  const int nthreads = blockDim.x;
-  const int warp = threadIdx.x >> 5;
-  const int nwarps = nthreads >> 5;
-
-  zero_sf_padding(sf, layout, M, C, Rp, Cp);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  const int64_t first = blockIdx.x;
-  const int64_t step = gridDim.x;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < stages; ++s) {
-      const int64_t r = first + s * step;
-      if (r < M) {
-        mbar_arrive_expect_tx(&full[s], row_bytes);
-        bulk_g2s(smem + static_cast<size_t>(s) * row_bytes, x + r * ldx, row_bytes, &full[s]);
-      }
+__device__ __forceinline__ void load_row_blocks(const uint16_t *xrow, int C, int nt, bool v8,
+                                                uint32_t (&w)[BPT][8]) {
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) {
+    const int c = static_cast<int>(threadIdx.x) + i * nt;
+    if (c < C) {
+      if (v8) ld_block16<true>(xrow + c * 16, w[i]);
+      else ld_block16<false>(xrow + c * 16, w[i]);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w[i][k] = 0u;  // zero blocks: amax 0, scale code 0
     }
   }
-  int stage = 0;
-  uint32_t parity = 0;
-  uint32_t j = 0;
-  for (int64_t r = first; r < M; r += step, ++j) {
-    const bool ok = mbar_wait_bounded(&full[stage], parity, kWaitTimeoutNs);
-    const uint8_t *row = smem + static_cast<size_t>(stage) * row_bytes;
+}
 
-    uint32_t w[BPT][8];
+template <int DTYPE, int BPT, int NT, int MINB>
+__global__ void __launch_bounds__(NT, MINB) quant_pertoken_regs_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t K, int64_t ldx, float *__restrict__ g,
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp, int64_t Cp,
+    bool v8) {
+  __shared__ float red[2][NT / 32];
+  const int C = static_cast<int>(K / 16);
+  const int warp = threadIdx.x >> 5;
+
+  uint32_t w[BPT][8];
+  int64_t r = blockIdx.x;
+  const int64_t step = gridDim.x;
+  if (r < M) load_row_blocks<DTYPE, BPT>(x + r * ldx, C, NT, v8, w);
+  zero_sf_padding(sf, layout, M, C, Rp, Cp);
+
+  for (uint32_t j = 0; r < M; r += step, ++j) {
     float bam[BPT];
     float m = 0.0f;
 #pragma unroll
     for (int i = 0; i < BPT; ++i) {
-      const int c = threadIdx.x + i * nthreads;
-      bam[i] = 0.0f;
-      if (c < C) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(row + c * 32);
-        const uint4 a = p[0], b = p[1];
-        w[i][0] = a.x; w[i][1] = a.y; w[i][2] = a.z; w[i][3] = a.w;
-        w[i][4] = b.x; w[i][5] = b.y; w[i][6] = b.z; w[i][7] = b.w;
-        bam[i] = amax16_packed<DTYPE>(w[i]);
-        m = fmaxf(m, bam[i]);
-      }
+      bam[i] = amax16_packed<DTYPE>(w[i]);
+      m = fmaxf(m, bam[i]);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    // red is double-buffered by row parity: row j + 2 writes this half only after every
+    // thread has passed row j + 1's barrier, i.e. after all reads of row j's partials.
     if (lane_id() == 0) red[j & 1][warp] = m;
-    // One barrier per row: row-maximum partials are visible, every thread is done reading the
-    // slot, and a timed-out wait anywhere makes the whole CTA leave together.
-    if (__syncthreads_or(!ok)) {
-      if (threadIdx.x == 0) atomicOr(&g_device_error, kDevErrTimeout);
-      return;
-    }
-    if (threadIdx.x == 0) {
-      const int64_t rn = r + static_cast<int64_t>(stages) * step;
-      if (rn < M) {
-        mbar_arrive_expect_tx(&full[stage], row_bytes);
-        bulk_g2s(smem + static_cast<size_t>(stage) * row_bytes, x + rn * ldx, row_bytes,
-                 &full[stage]);
-      }
-    }
+    __syncthreads();
     float amax = red[j & 1][0];
-    for (int w2 = 1; w2 < nwarps; ++w2) amax = fmaxf(amax, red[j & 1][w2]);
+#pragma unroll
+    for (int w2 = 1; w2 < NT / 32; ++w2) amax = fmaxf(amax, red[j & 1][w2]);
     const float gr = global_scale_from_amax(amax);
     if (threadIdx.x == 0) g[r] = gr;
     const float tab = row_recip_lane(gr);
 
     uint8_t *qrow = q + r * (K / 2);
     uint8_t *sfrow = sf + sf_row_base(layout, r, C, Cp);
+    const int64_t rn = r + step;
+    const uint16_t *xn = x + rn * ldx;
 #pragma unroll
     for (int i = 0; i < BPT; ++i) {
-      const int c = threadIdx.x + i * nthreads;
-      // out-of-row slots carry bam = 0 (code 0) and still join the table shuffle
+      const int c = static_cast<int>(threadIdx.x) + i * NT;
+      // out-of-row slots carry zero blocks (code 0) and still join the table shuffle
       const uint32_t s = block_scale_code(bam[i], gr);
       const float rr = row_recip(s, tab);
       if (c < C) {
         st_cs_u64(qrow + c * 8, quant_packed16<DTYPE>(w[i], rr));
         sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);
+        if (rn < M) {
+          if (v8) ld_block16<true>(xn + c * 16, w[i]);
+          else ld_block16<false>(xn + c * 16, w[i]);
+        }
       }
-    }
-    if (++stage == stages) {
-      stage = 0;
-      parity ^= 1u;
     }
   }
 }
@@ -622,61 +599,29 @@ cudaError_t launch_quantize(const void *x, int dtype, int64_t M, int64_t K, int6
                              xp, M, K, ldx, g, 0, q, sf, layout, Rp, Cp)));
     return cudaGetLastError();
   }
-  const int64_t row_bytes = K * 2;
   const int C = static_cast<int>(K / 16);
-  // Blocks per thread: the smallest power of two that keeps a row within 128 threads
-  // (within 256 once 8 blocks per thread no longer suffice). Four blocks per thread on a
-  // 128-thread CTA was the fastest shape measured for 7168-wide rows: fewer CTA barriers
-  // per row than 2 x 224 threads, more rows in flight than one warp per row.
-  int bpt = 1;
-  while (bpt < 8 && (static_cast<int64_t>(C) + bpt - 1) / bpt > 128) bpt *= 2;
-  if ((static_cast<int64_t>(C) + bpt - 1) / bpt > 256) bpt = 16;
-  int stages = 0, per_sm = 0;
-  int nthreads = 0;
-  if (bpt <= 8) {
-    nthreads = static_cast<int>(((C + bpt - 1) / bpt + 31) / 32 * 32);
-    // Rows in flight per SM = CTAs per SM x stages, within ~220 KB of shared memory and
-    // 2048 threads per SM; prefer more CTAs on a tie.
-    for (int s = 2; s <= 4 && s <= kRowcacheMaxStages; ++s) {
-      const int64_t smem = row_bytes * s + 1024;
-      if (smem > max_smem_optin) break;
-      int cps = static_cast<int>((220 * 1024) / smem);
-      if (cps > 2048 / nthreads) cps = 2048 / nthreads;
-      if (cps > 32) cps = 32;
-      if (cps >= 1 && cps * s > per_sm * stages) {
-        stages = s;
-        per_sm = cps;
-      }
-    }
-  }
-  if (stages >= 2) {
-    const size_t smem = static_cast<size_t>(row_bytes * stages);
-    int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
-    if (grid > M) grid = M;
-    if (grid < 1) grid = 1;
-#define NVFP4_LAUNCH_ROWCACHE(DT, B)                                                          \
-  do {                                                                                        \
-    cudaError_t e = cudaFuncSetAttribute(quant_pertoken_rowcache_kernel<DT, B>,               \
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,         \
-                                         static_cast<int>(smem));                             \
-    if (e != cudaSuccess) return e;                                                           \
-    quant_pertoken_rowcache_kernel<DT, B><<<static_cast<int>(grid), nthreads, smem, st>>>(   \
-        xp, M, K, ldx, g, q, sf, layout, Rp, Cp, stages);                                     \
+  // A row lives in the registers of one CTA: 128 threads with 1, 2, 4 or 8 blocks each up to
+  // 1024 blocks per row (K = 16384), 256 threads with 4 or 8 blocks each up to 2048
+  // (K = 32768). The grid is the number of CTAs the launch bounds guarantee resident.
+#define NVFP4_LAUNCH_REGS(B, NT, MINB)                                                          \
+  do {                                                                                          \
+    int64_t cg = static_cast<int64_t>(num_sms) * (MINB);                                        \
+    if (cg > M) cg = M;                                                                         \
+    if (cg < 1) cg = 1;                                                                         \
+    if (dtype == kInBf16)                                                                       \
+      quant_pertoken_regs_kernel<0, B, NT, MINB><<<static_cast<int>(cg), NT, 0, st>>>(          \
+          xp, M, K, ldx, g, q, sf, layout, Rp, Cp, v8);                                         \
+    else                                                                                        \
+      quant_pertoken_regs_kernel<1, B, NT, MINB><<<static_cast<int>(cg), NT, 0, st>>>(          \
+          xp, M, K, ldx, g, q, sf, layout, Rp, Cp, v8);                                         \
+    return cudaGetLastError();                                                                  \
   } while (0)
-    if (dtype == kInBf16) {
-      if (bpt == 1) NVFP4_LAUNCH_ROWCACHE(0, 1);
-      else if (bpt == 2) NVFP4_LAUNCH_ROWCACHE(0, 2);
-      else if (bpt == 4) NVFP4_LAUNCH_ROWCACHE(0, 4);
-      else NVFP4_LAUNCH_ROWCACHE(0, 8);
-    } else {
-      if (bpt == 1) NVFP4_LAUNCH_ROWCACHE(1, 1);
-      else if (bpt == 2) NVFP4_LAUNCH_ROWCACHE(1, 2);
-      else if (bpt == 4) NVFP4_LAUNCH_ROWCACHE(1, 4);
-      else NVFP4_LAUNCH_ROWCACHE(1, 8);
-    }
-#undef NVFP4_LAUNCH_ROWCACHE
-    return cudaGetLastError();
-  }
+  if (C <= 128) NVFP4_LAUNCH_REGS(1, 128, 8);
+  if (C <= 256) NVFP4_LAUNCH_REGS(2, 128, 8);
+  if (C <= 512) NVFP4_LAUNCH_REGS(4, 128, 8);
+  if (C <= 1024) NVFP4_LAUNCH_REGS(8, 128, 4);
+  if (C <= 2048) NVFP4_LAUNCH_REGS(8, 256, 2);
+#undef NVFP4_LAUNCH_REGS
   // Rows too long to stage: row amax pass, then the streaming pass with per-row g.
   const int rgrid = static_cast<int>(M < num_sms * 8 ? M : num_sms * 8);
   const int threads = row_threads(K / 16, 2);

@@ -55,6 +55,18 @@ def test_quantize_parity_small(M, K, pad, layout, per_token, dtype):
     _quantize_both(nv, xt, dtype, per_token, layout, K)
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("M,K,pad", [(1300, 4096, 8), (700, 16384, 0), (350, 20480, 8),
+                                     (40, 32768, 0), (9, 32784, 0)])
+def test_quantize_per_token_row_shapes(M, K, pad, dtype):
+    # every register-resident row shape (1, 2, 4, 8 blocks per thread; 128 and 256 threads),
+    # more rows than resident CTAs so rows roll through the registers, rows whose stride is
+    # not a multiple of 32 bytes, and the first K past the register path (two-pass)
+    nv = require_cuda()
+    xt = _inputs(M, K, pad, seed=M + 7 * K, dtype=dtype)
+    _quantize_both(nv, xt, dtype, True, 1, K)
+
+
 def test_quantize_per_token_long_rows_two_pass():
     # rows of 65536 elements (128 KB) do not fit twice in shared memory: two-pass path
     nv = require_cuda()
