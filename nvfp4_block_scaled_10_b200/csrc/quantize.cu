@@ -20,6 +20,7 @@
 
 #include "kernels.h"
 #include "ptx.cuh"
+#include "swiglu_math.cuh"
 
 namespace nvfp4 {
 
@@ -396,43 +397,23 @@ __global__ void __launch_bounds__(NT, MINB) quant_pertoken_regs_kernel(
 
 // ------------------------------------------------------------------------------ SwiGLU
 
-// Library fp32 exponential on a pair of values: clamp to [-87, 88]; k = rint(v * log2 e);
-// Cody-Waite reduction f = v - k*ln2_hi - k*ln2_lo; degree-7 Taylor polynomial of e^f
-// (coefficients 1/n! rounded to fp32) by fused multiply-add; times 2^k built from exponent
-// bits. Packed fp32x2 instructions give each lane the same IEEE results as scalar code.
-// rint is taken as (z + 1.5*2^23) - 1.5*2^23: for |z| < 2^22 the sum is rounded to an
-// integer with ties to even, which is exactly rint(z), and its low mantissa bits are k.
-__device__ __forceinline__ F2 exp2_f32(F2 v) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  v.x = fminf(fmaxf(v.x, -87.0f), 88.0f);
-  v.y = fminf(fmaxf(v.y, -87.0f), 88.0f);
-  const F2 z = mul2f_rn(v, F2{0x1.715476p+0f, 0x1.715476p+0f});
-  const F2 t = add2f_rn(z, F2{kRound, kRound});
-  const F2 k = add2f_rn(t, F2{-kRound, -kRound});
-  const F2 nk{-k.x, -k.y};
-  F2 f = fma2_rn(nk, F2{0x1.62e4p-1f, 0x1.62e4p-1f}, v);
-  f = fma2_rn(nk, F2{0x1.7f7d1cp-20f, 0x1.7f7d1cp-20f}, f);
-  F2 p{0x1.a01a02p-13f, 0x1.a01a02p-13f};                   // 1/7!
-  p = fma2_rn(p, f, F2{0x1.6c16c2p-10f, 0x1.6c16c2p-10f});  // 1/6!
-  p = fma2_rn(p, f, F2{0x1.111112p-7f, 0x1.111112p-7f});    // 1/5!
-  p = fma2_rn(p, f, F2{0x1.555556p-5f, 0x1.555556p-5f});    // 1/4!
-  p = fma2_rn(p, f, F2{0x1.555556p-3f, 0x1.555556p-3f});    // 1/3!
-  p = fma2_rn(p, f, F2{0.5f, 0.5f});                        // 1/2!
-  p = fma2_rn(p, f, F2{1.0f, 1.0f});                        // 1/1!
-  p = fma2_rn(p, f, F2{1.0f, 1.0f});                        // 1/0!
-  // 2^k: k sits in the low bits of t (t's bits = 0x4B400000 + k), so (k + 127) << 23 is
-  // (bits(t) - 0x4B400000 + 127) << 23.
-  const F2 two_k{__int_as_float((__float_as_int(t.x) - 0x4B3FFF81) << 23),
-                 __int_as_float((__float_as_int(t.y) - 0x4B3FFF81) << 23)};
-  return mul2f_rn(p, two_k);
-}
-
-// y = silu(gate) * up = gate / (1 + e(-gate)) * up for a pair of elements.
-__device__ __forceinline__ F2 swiglu2_f32(F2 gate, F2 up) {
-  const F2 e = exp2_f32(F2{-gate.x, -gate.y});
-  const F2 den = add2f_rn(F2{1.0f, 1.0f}, e);
-  const F2 silu{__fdiv_rn(gate.x, den.x), __fdiv_rn(gate.y, den.y)};
-  return mul2f_rn(silu, up);
+// y = silu(gate) * up for the 16 elements of one block (8 packed words of each half);
+// returns max |y|.
+template <int DTYPE, bool SAFE>
+__device__ __forceinline__ float swiglu_block16(const uint32_t (&wg)[8], const uint32_t (&wu)[8],
+                                                float (&y)[16]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    F2 gate, up;
+    unpack2<DTYPE>(wg[i], gate.x, gate.y);
+    unpack2<DTYPE>(wu[i], up.x, up.y);
+    const F2 v = swiglu2_f32<SAFE>(gate, up);
+    y[2 * i] = v.x;
+    y[2 * i + 1] = v.y;
+    amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+  }
+  return amax;
 }
 
 // Row-major like quant_stream_kernel: CTA b handles rows b, b + gridDim.x, ...; thread t
@@ -468,17 +449,11 @@ __global__ void __launch_bounds__(256) swiglu_quant_kernel(
         const int c = c0 + u * blockDim.x;
         if (c < C) {
           float y[16];
-          float amax = 0.0f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            F2 gate, up;
-            unpack2<DTYPE>(wg[u][i], gate.x, gate.y);
-            unpack2<DTYPE>(wu[u][i], up.x, up.y);
-            const F2 v = swiglu2_f32(gate, up);
-            y[2 * i] = v.x;
-            y[2 * i + 1] = v.y;
-            amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
-          }
+          float amax;
+          // an infinite gate needs the quotient's special-value select; NaN and finite
+          // gates do not (the packed maximum skips NaN, so it is infinite only for +-inf)
+          if (amax16_packed<DTYPE>(wg[u]) != INFINITY) amax = swiglu_block16<DTYPE, false>(wg[u], wu[u], y);
+          else amax = swiglu_block16<DTYPE, true>(wg[u], wu[u], y);
           const uint32_t s = block_scale_code(amax, g0);
           st_cs_u64(qrow + c * 8, quant_f32x16(y, rtab[s]));
           sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);

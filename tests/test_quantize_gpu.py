@@ -169,6 +169,28 @@ def test_swiglu_extreme_gates():
         assert_bytes_equal(host_bytes(sf), sf_o, "sf")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_swiglu_infinite_and_signed_zero_gates(dtype):
+    # blocks holding an infinite gate take the kernel's exact-special-value quotient; the
+    # neighbouring blocks (finite gates, -0 among them) take the form without it
+    nv = require_cuda()
+    tdt, odt = DT[dtype]
+    inf = float("inf")
+    gate = torch.tensor([[inf, -inf, -0.0, 0.0, 1.5, -2.0, 3.0, -0.25, 7.0, -7.0, 0.5, 1.0,
+                          -1.0, 2.0, -3.0, 4.0] + [-0.0, 0.0, 0.125, -0.125] * 4,
+                         [-inf] + [0.5] * 15 + [inf] + [-0.5] * 15], dtype=torch.float32)
+    up = torch.linspace(0.5, 3.0, 32).reshape(1, 32).repeat(2, 1)
+    x = torch.cat([gate, up], dim=1).to(tdt)
+    bits = workloads.bits16(x)
+    for g in [1.0, 37.5]:
+        q_o, sf_o = orc.swiglu_quantize(bits, g, odt)
+        q, sf = nv.swiglu_nvfp4_quantize(x.cuda(), torch.tensor([g], device="cuda"),
+                                         sf_layout=nv.SF_LINEAR)
+        torch.cuda.synchronize()
+        assert_bytes_equal(host_bytes(q), q_o, "q")
+        assert_bytes_equal(host_bytes(sf), sf_o, "sf")
+
+
 @pytest.mark.parametrize("layout", [0, 1, 2])
 @pytest.mark.parametrize("R,C", [(1, 1), (130, 7), (300, 33), (28672, 512)])
 def test_swizzle_unswizzle_parity(R, C, layout):
