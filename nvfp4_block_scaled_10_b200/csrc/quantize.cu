@@ -399,16 +399,15 @@ __global__ void __launch_bounds__(NT, MINB) quant_pertoken_regs_kernel(
 
 // y = silu(gate) * up for the 16 elements of one block (8 packed words of each half);
 // returns max |y|.
-template <int DTYPE, bool SAFE>
+template <int DTYPE, bool CLAMP, bool SAFE>
 __device__ __forceinline__ float swiglu_block16(const uint32_t (&wg)[8], const uint32_t (&wu)[8],
                                                 float (&y)[16]) {
   float amax = 0.0f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    F2 gate, up;
-    unpack2<DTYPE>(wg[i], gate.x, gate.y);
+    F2 up;
     unpack2<DTYPE>(wu[i], up.x, up.y);
-    const F2 v = swiglu2_f32<SAFE>(gate, up);
+    const F2 v = mul2f_rn(silu_pair_neg<CLAMP, SAFE>(unpack2_neg<DTYPE>(wg[i])), up);
     y[2 * i] = v.x;
     y[2 * i + 1] = v.y;
     amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
@@ -416,50 +415,83 @@ __device__ __forceinline__ float swiglu_block16(const uint32_t (&wg)[8], const u
   return amax;
 }
 
-// Row-major like quant_stream_kernel: CTA b handles rows b, b + gridDim.x, ...; thread t
-// owns blocks t, t + blockDim.x, ... of the output row (gate and up loaded as two 32-byte
-// blocks each).
+// Persistent: the work items are (row, chunk) pairs, a chunk being NT * UNROLL consecutive
+// output blocks of a row, dealt round-robin to the CTAs (the row count of the workloads is
+// not a multiple of the grid, so whole rows would leave a long tail). Thread t owns blocks
+// t + u * NT (u < UNROLL) of the chunk; gate and up are loaded as two 32-byte blocks each.
+// Once y of block u is formed, block u of the CTA's next item is loaded into the registers
+// it held, so the next item streams in while this one is quantized. Per block the packed
+// maximum |gate| picks the cheapest silu form that is exact for it.
 template <int DTYPE, int UNROLL, bool V8>
-__global__ void __launch_bounds__(256) swiglu_quant_kernel(
+__device__ __forceinline__ void load_swiglu_item(const uint16_t *x, int64_t ldx, int64_t H, int C,
+                                                 int64_t r, int c0, int nt, uint32_t (&wg)[UNROLL][8],
+                                                 uint32_t (&wu)[UNROLL][8]) {
+  const uint16_t *grow = x + r * ldx;
+#pragma unroll
+  for (int u = 0; u < UNROLL; ++u) {
+    const int c = c0 + u * nt;
+    if (c < C) {
+      ld_block16<V8>(grow + c * 16, wg[u]);
+      ld_block16<V8>(grow + H + c * 16, wu[u]);
+    }
+  }
+}
+
+template <int DTYPE, int UNROLL, bool V8, int NT, int MINB>
+__global__ void __launch_bounds__(NT, MINB) swiglu_quant_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t H, int64_t ldx, const float *__restrict__ g,
-    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp, int64_t Cp) {
+    uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp, int64_t Cp,
+    int chunks_per_row) {
   __shared__ float rtab[128];
   const int C = static_cast<int>(H / 16);
   const float g0 = g[0];
+  // item = blockIdx.x + k * gridDim.x as (row r, chunk ch), advanced without a division
+  const int64_t step_r = gridDim.x / chunks_per_row;
+  const int step_ch = static_cast<int>(gridDim.x % chunks_per_row);
+  int64_t r = blockIdx.x / chunks_per_row;
+  int ch = static_cast<int>(blockIdx.x % chunks_per_row);
+  uint32_t wg[UNROLL][8], wu[UNROLL][8];
+  if (r < M) load_swiglu_item<DTYPE, UNROLL, V8>(x, ldx, H, C, r, ch * (NT * UNROLL) + threadIdx.x, NT, wg, wu);
   fill_recip_table(rtab, g0);
   __syncthreads();
-  const int step = blockDim.x * UNROLL;
-  for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
-    const uint16_t *grow = x + r * ldx;
-    const uint16_t *urow = grow + H;
+  while (r < M) {
+    int64_t rn = r + step_r;
+    int chn = ch + step_ch;
+    if (chn >= chunks_per_row) {
+      chn -= chunks_per_row;
+      ++rn;
+    }
+    const int c0 = ch * (NT * UNROLL) + static_cast<int>(threadIdx.x);
+    const int c0n = chn * (NT * UNROLL) + static_cast<int>(threadIdx.x);
+    const uint16_t *gnext = x + rn * ldx;
     uint8_t *qrow = q + r * (H / 2);
     uint8_t *sfrow = sf + sf_row_base(layout, r, C, Cp);
-    for (int c0 = threadIdx.x; c0 < C; c0 += step) {
-      uint32_t wg[UNROLL][8], wu[UNROLL][8];
 #pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        const int c = c0 + u * blockDim.x;
-        if (c < C) {
-          ld_block16<V8>(grow + c * 16, wg[u]);
-          ld_block16<V8>(urow + c * 16, wu[u]);
-        }
+    for (int u = 0; u < UNROLL; ++u) {
+      const int c = c0 + u * NT;
+      float y[16];
+      float amax = 0.0f;
+      if (c < C) {
+        // the packed maximum skips NaN: it exceeds 87 only for a gate beyond the exp clamp
+        // and is infinite only for an infinite gate
+        const float gmax = amax16_packed<DTYPE>(wg[u]);
+        if (gmax <= 87.0f) amax = swiglu_block16<DTYPE, false, false>(wg[u], wu[u], y);
+        else if (gmax != INFINITY) amax = swiglu_block16<DTYPE, true, false>(wg[u], wu[u], y);
+        else amax = swiglu_block16<DTYPE, true, true>(wg[u], wu[u], y);
       }
-#pragma unroll
-      for (int u = 0; u < UNROLL; ++u) {
-        const int c = c0 + u * blockDim.x;
-        if (c < C) {
-          float y[16];
-          float amax;
-          // an infinite gate needs the quotient's special-value select; NaN and finite
-          // gates do not (the packed maximum skips NaN, so it is infinite only for +-inf)
-          if (amax16_packed<DTYPE>(wg[u]) != INFINITY) amax = swiglu_block16<DTYPE, false>(wg[u], wu[u], y);
-          else amax = swiglu_block16<DTYPE, true>(wg[u], wu[u], y);
-          const uint32_t s = block_scale_code(amax, g0);
-          st_cs_u64(qrow + c * 8, quant_f32x16(y, rtab[s]));
-          sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);
-        }
+      const int cn = c0n + u * NT;
+      if (rn < M && cn < C) {
+        ld_block16<V8>(gnext + cn * 16, wg[u]);
+        ld_block16<V8>(gnext + H + cn * 16, wu[u]);
+      }
+      if (c < C) {
+        const uint32_t s = block_scale_code(amax, g0);
+        st_cs_u64(qrow + c * 8, quant_f32x16(y, rtab[s]));
+        sfrow[sf_col_off(layout, c)] = static_cast<uint8_t>(s);
       }
     }
+    r = rn;
+    ch = chn;
   }
   zero_sf_padding(sf, layout, M, C, Rp, Cp);
 }
@@ -612,12 +644,19 @@ cudaError_t launch_swiglu_quantize(const void *x, int dtype, int64_t M, int64_t 
                                    const float *g, uint8_t *q, uint8_t *sf, int layout, int64_t Rp,
                                    int64_t Cp, int num_sms, cudaStream_t st) {
   const uint16_t *xp = static_cast<const uint16_t *>(x);
-  const int threads = row_threads(H / 16, 2);
-  const int grid = row_grid(M, threads, num_sms);
+  // 224 threads x 2 blocks: a 14336-wide output row (896 blocks) is two chunks. Four CTAs per
+  // SM are resident (launch bounds), and the grid is exactly that many.
+  constexpr int kNT = 224, kUnroll = 2, kMinB = 4;
+  const int64_t C = H / 16;
+  const int cpr = static_cast<int>((C + kNT * kUnroll - 1) / (kNT * kUnroll));
+  int64_t grid = static_cast<int64_t>(num_sms) * kMinB;
+  if (grid > M * cpr) grid = M * cpr;
+  if (grid < 1) grid = 1;
   const bool v8 = blocks_32b_aligned(x, ldx);
   NVFP4_DISPATCH_DT_V8(dtype, v8,
-                       (swiglu_quant_kernel<DT, 2, VV><<<grid, threads, 0, st>>>(
-                           xp, M, H, ldx, g, q, sf, layout, Rp, Cp)));
+                       (swiglu_quant_kernel<DT, kUnroll, VV, kNT, kMinB>
+                        <<<static_cast<int>(grid), kNT, 0, st>>>(xp, M, H, ldx, g, q, sf, layout,
+                                                                 Rp, Cp, cpr)));
   return cudaGetLastError();
 }
 

@@ -187,7 +187,8 @@ uint16_t orc_f64_to_f16(double v) {
 /* The pages fix SwiGLU to fp32 registers but not an exp; bit-exact quantized output      */
 /* needs one exact definition on both sides. Written from the mathematics:                */
 /*   x clamped to [-87, 88] (keeps 2^k a normal number),                                  */
-/*   k = rint(x * log2(e)) (fp32 product, round half to even),                            */
+/*   k = the integer nearest the exact product x * fl(log2 e), ties to even (the product  */
+/*       of two fp32 values is exact in double, so it is formed there and rounded once),  */
 /*   f = x - k*ln2 with ln2 split hi/lo (Cody & Waite, "Software Manual for the           */
 /*       Elementary Functions", 1980): hi = 0x3F317200 has 15 significant bits, so k*hi  */
 /*       is exact for |k| <= 127,                                                         */
@@ -214,8 +215,8 @@ static const float ORC_INV_FACT[8] = {
 float orc_exp(float x) {
   if (x < -87.0f) x = -87.0f;
   if (x > 88.0f) x = 88.0f;
-  float z = x * ORC_LOG2E;
-  float k = rintf(z); /* default rounding mode: to nearest, ties to even */
+  double z = (double)x * (double)ORC_LOG2E; /* exact: 24 x 24 significant bits */
+  float k = (float)rint(z);                  /* default rounding: to nearest, ties to even */
   float f = fmaf(-k, ORC_LN2_HI, x);
   f = fmaf(-k, ORC_LN2_LO, f);
   float p = ORC_INV_FACT[7];

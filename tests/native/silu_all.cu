@@ -10,20 +10,14 @@
 
 namespace {
 
-template <bool SAFE>
+template <bool CLAMP, bool SAFE>
 __global__ void silu_kernel(const uint16_t *__restrict__ bits, int dtype, int n, float *__restrict__ out) {
   const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (i >= n) return;
-  nvfp4::F2 gate;
-  const uint16_t b0 = bits[i], b1 = (i + 1 < n) ? bits[i + 1] : 0;
-  if (dtype == 0) {
-    gate.x = __uint_as_float(static_cast<uint32_t>(b0) << 16);
-    gate.y = __uint_as_float(static_cast<uint32_t>(b1) << 16);
-  } else {
-    gate.x = __half2float(__ushort_as_half(b0));
-    gate.y = __half2float(__ushort_as_half(b1));
-  }
-  const nvfp4::F2 s = nvfp4::silu2_f32<SAFE>(gate);
+  const uint32_t b0 = bits[i], b1 = (i + 1 < n) ? bits[i + 1] : 0;
+  const uint32_t w = b0 | (b1 << 16);
+  const nvfp4::F2 v = dtype == 0 ? nvfp4::unpack2_neg<0>(w) : nvfp4::unpack2_neg<1>(w);
+  const nvfp4::F2 s = nvfp4::silu_pair_neg<CLAMP, SAFE>(v);
   out[i] = s.x;
   if (i + 1 < n) out[i + 1] = s.y;
 }
@@ -31,8 +25,8 @@ __global__ void silu_kernel(const uint16_t *__restrict__ bits, int dtype, int n,
 }  // namespace
 
 // Returns 0 on success, else the CUDA error code. host_bits: n gates; host_out: n floats.
-// safe = 1 runs the form with the infinite-dividend select, 0 the form without it.
-extern "C" int silu_all(const uint16_t *host_bits, int dtype, int n, float *host_out, int safe) {
+// form 0: no clamp, no infinite-dividend select; 1: clamp only; 2: clamp and select.
+extern "C" int silu_all(const uint16_t *host_bits, int dtype, int n, float *host_out, int form) {
   uint16_t *d_bits = nullptr;
   float *d_out = nullptr;
   cudaError_t e = cudaMalloc(&d_bits, n * sizeof(uint16_t));
@@ -40,8 +34,10 @@ extern "C" int silu_all(const uint16_t *host_bits, int dtype, int n, float *host
   if (e == cudaSuccess) e = cudaMemcpy(d_bits, host_bits, n * sizeof(uint16_t), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) {
     const int pairs = (n + 1) / 2;
-    if (safe) silu_kernel<true><<<(pairs + 255) / 256, 256>>>(d_bits, dtype, n, d_out);
-    else silu_kernel<false><<<(pairs + 255) / 256, 256>>>(d_bits, dtype, n, d_out);
+    const int grid = (pairs + 255) / 256;
+    if (form == 0) silu_kernel<false, false><<<grid, 256>>>(d_bits, dtype, n, d_out);
+    else if (form == 1) silu_kernel<true, false><<<grid, 256>>>(d_bits, dtype, n, d_out);
+    else silu_kernel<true, true><<<grid, 256>>>(d_bits, dtype, n, d_out);
     e = cudaGetLastError();
   }
   if (e == cudaSuccess) e = cudaMemcpy(host_out, d_out, n * sizeof(float), cudaMemcpyDeviceToHost);

@@ -34,21 +34,27 @@ def silu_lib(tmp_path_factory):
     return lib
 
 
-@pytest.mark.parametrize("safe", [True, False])
+@pytest.mark.parametrize("form", [0, 1, 2])
 @pytest.mark.parametrize("dtype", [orc.BF16, orc.FP16])
-def test_silu_every_gate_matches_oracle(silu_lib, dtype, safe):
-    # the kernel takes the form without the infinite-dividend select for blocks with no
-    # infinite gate: that form is checked on every gate but the two infinities
+def test_silu_every_gate_matches_oracle(silu_lib, dtype, form):
+    # the kernel picks a form per block from the block's largest |gate| (NaN skipped):
+    # form 0 (no exp clamp, no infinite-dividend select) for |gate| <= 87, form 1 (clamp)
+    # for other finite gates, form 2 (clamp and select) when a gate is infinite. Each form
+    # is checked on every gate it can meet, NaN included.
     bits = np.arange(1 << 16, dtype=np.uint16)
     if dtype == orc.BF16:
         gate = (bits.astype(np.uint32) << 16).view(np.float32)
     else:
         gate = orc.f16_to_f32(bits)
-    if not safe:
+    if form == 0:
+        keep = np.isnan(gate) | (np.abs(gate) <= 87.0)
+    elif form == 1:
         keep = ~np.isinf(gate)
-        bits, gate = bits[keep], gate[keep]
+    else:
+        keep = np.ones(gate.shape, bool)
+    bits, gate = bits[keep], gate[keep]
     out = np.empty(bits.size, np.float32)
-    rc = silu_lib.silu_all(bits.ctypes.data, int(dtype), bits.size, out.ctypes.data, int(safe))
+    rc = silu_lib.silu_all(bits.ctypes.data, int(dtype), bits.size, out.ctypes.data, int(form))
     assert rc == 0, f"CUDA error {rc}"
     ref = orc.silu32(gate)
     both_nan = np.isnan(out) & np.isnan(ref)
