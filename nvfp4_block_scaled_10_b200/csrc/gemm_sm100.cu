@@ -32,6 +32,7 @@
 // tokens its N = BN columns) so the weight stream fills the MMA.
 #include <cfloat>
 #include <cstdint>
+#include <mutex>
 
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -136,6 +137,7 @@ struct KernelParams {
   const uint8_t *sfb;  // scales of the MMA B operand (128x4, or 8x4 when sfb_8x4)
   int sfb_8x4;
   int64_t sfb_rows_padded;  // rows of the B-scale buffer
+  int64_t sfa_rows_padded;  // rows of the A-scale buffer
   const float *ga;
   const float *gw;
   __half *out;
@@ -291,6 +293,7 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * C::kAccCols;
+        int prev = -1;  // stage whose release (commit) is still to be issued
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int stage = static_cast<int>(it % STAGES);
           const uint32_t round = it / STAGES;
@@ -301,6 +304,11 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
             break;
           }
           tc_fence_after();
+          // Release the previous stage only now: a barrier wait issued after a commit holds
+          // this thread until that commit's MMAs have completed, so committing stage s before
+          // waiting for stage s + 1 would leave the tensor pipe empty in between. Committed
+          // here, the wait above overlaps the previous stage's MMAs.
+          if (prev >= 0) tc_commit(&empty[prev]);
           const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
           const uint32_t sA = smem_u32(smem + C::kOffA + stage * C::kABytes);
           const uint32_t sB = smem_u32(smem + C::kOffB + stage * C::kBBytes);
@@ -311,8 +319,9 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
                      slot + kK64PerStage * C::kSfaColsPerK64 + a * C::kSfbColsPerK64,
                      (kt | a) != 0 ? 1u : 0u);
           }
-          tc_commit(&empty[stage]);
+          prev = stage;
         }
+        if (prev >= 0) tc_commit(&empty[prev]);
         if (ok) tc_commit(&acc_full[buf]);
       }
     }
@@ -450,6 +459,313 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------ CTA pairs
+
+// Large-M form: a cluster of two CTAs computes a 256 x 256 tile with the pair MMA
+// (tcgen05.mma.cta_group::2, M = 256, N = 256). CTA r of the pair holds rows
+// [128 r, 128 r + 128) of the tile's A and of its B (each CTA stages half of B), and its
+// tensor memory holds its 128 accumulator rows for all 256 columns, so every byte staged in a
+// CTA feeds twice the MMA work of the single-CTA 128 x 256 tile (a third less L2 -> SM
+// traffic per FLOP). Each CTA keeps the scales its half of the MMA reads in its own tensor
+// memory: A's for its 128 rows and B's for all 256 (same lane/column layout as the
+// single-CTA N = 256 case).
+//
+// Synchronisation (barriers named by the CTA holding them):
+//   full[s]      even CTA; both producers arrive.expect_tx and both CTAs' tile copies
+//                complete on it (count 2)
+//   sf_ready[s]  each CTA; its own scale atoms landed (count 1, bulk copies)
+//   sf_full[s]   even CTA; the four scale warps of both CTAs wrote their tensor memory
+//                (count 8)
+//   empty[s]     each CTA; pair-MMA commit multicast to both CTAs
+//   acc_full     each CTA; pair-MMA commit multicast after a tile's last MMA
+//   acc_empty    even CTA; the epilogue warps of both CTAs drained the accumulator (count 16)
+// Every wait is bounded; a cluster barrier opens and closes the kernel so no CTA touches its
+// peer's shared memory before the peer initialised it or after the peer exited.
+template <int STAGES>
+struct PairCfg {
+  static constexpr int kN = 256;                        // MMA N (tile columns)
+  static constexpr int kHalf = 128;                     // rows of A and of B per CTA
+  static constexpr int kABytes = kHalf * kBKBytes;      // 16 KB
+  static constexpr int kBBytes = kHalf * kBKBytes;      // 16 KB
+  static constexpr int kSfaBytes = kK64PerStage * kSfAtomBytes;      // 2 KB
+  static constexpr int kSfbBytes = 2 * kK64PerStage * kSfAtomBytes;  // 4 KB (all 256 rows)
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + STAGES * kABytes;
+  static constexpr int kOffSfa = kOffB + STAGES * kBBytes;
+  static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
+  static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
+  // full[S], sf_ready[S], sf_full[S], empty[S], acc_full, acc_empty, tmem slot
+  static constexpr int kBarBytes = (4 * STAGES + 2) * 8 + 16;
+  static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
+  static constexpr int kAccCols = kN;
+  static constexpr int kSfaColsPerK64 = 4;
+  static constexpr int kSfbColsPerK64 = 8;
+  static constexpr int kSlotCols = kK64PerStage * (kSfaColsPerK64 + kSfbColsPerK64);
+  static constexpr int kSfCol0 = kAccCols;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kColsPerEpiWarp = kN * 4 / kEpiWarps;  // 128
+  static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+  static_assert(kSfCol0 + STAGES * kSlotCols <= kTmemCols, "TMEM columns");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+  // kind::mxf4nvf4: E2M1 A and B, K-major, UE4M3 scales; N >> 3 at bit 17, M >> 4 at bit 24
+  static constexpr uint32_t kIdesc =
+      (1u << 7) | (1u << 10) | (uint32_t(kN >> 3) << 17) | (uint32_t(256 >> 4) << 24);
+};
+
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kThreads, 1)
+    gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                           const __grid_constant__ CUtensorMap tmap_b, const KernelParams p) {
+  using C = PairCfg<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+  uint64_t *sf_ready = full + STAGES;
+  uint64_t *sf_full = sf_ready + STAGES;
+  uint64_t *empty = sf_full + STAGES;
+  uint64_t *acc_full = empty + STAGES;
+  uint64_t *acc_empty = acc_full + 1;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int64_t K = p.K;
+  const int num_k64 = static_cast<int>(K / 64);
+  const int num_kt = (num_k64 + kK64PerStage - 1) / kK64PerStage;
+  const int64_t k64_per_row = K / 64;
+  const int num_tiles = p.tiles_a * p.tiles_b;  // tiles_a along M (256 rows), tiles_b along N
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int npairs = static_cast<int>(gridDim.x >> 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 2);
+      mbar_init(&sf_ready[s], 1);
+      mbar_init(&sf_full[s], 8);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * C::kEpiWarps);
+    fence_mbar_init();
+    prefetch_tmap(&tmap_a);
+    prefetch_tmap(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, C::kTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto tile_origin = [&](int t, int64_t &m0, int64_t &n0) {
+    m0 = static_cast<int64_t>(t % p.tiles_a) * 256;
+    n0 = static_cast<int64_t>(t / p.tiles_a) * C::kN;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer (each CTA)
+    uint32_t it = 0;
+    bool ok = true;
+    const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
+    for (int t = pair; t < num_tiles && ok; t += npairs) {
+      int64_t m0, n0;
+      tile_origin(t, m0, n0);
+      const int64_t arow = m0 + C::kHalf * rank;  // this CTA's A rows and B rows
+      const int64_t brow = n0 + C::kHalf * rank;
+      int sfb_copies = 0;
+      for (int blk = 0; blk < 2; ++blk)
+        if ((n0 / 128 + blk) * 128 < p.sfb_rows_padded) ++sfb_copies;
+      const bool sfa_copy = arow < p.sfa_rows_padded;
+      for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        const int stage = static_cast<int>(it % STAGES);
+        const uint32_t round = it / STAGES;
+        if (it >= STAGES) {
+          if (!mbar_wait_cluster_warp(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
+            if (lane == 0) report_timeout(p.dev_status);
+            ok = false;
+            break;
+          }
+        }
+        const int k64_0 = kt * kK64PerStage;
+        const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+        uint8_t *sA = smem + C::kOffA + stage * C::kABytes;
+        uint8_t *sB = smem + C::kOffB + stage * C::kBBytes;
+        uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
+        uint8_t *sSfb = smem + C::kOffSfb + stage * C::kSfbBytes;
+        if (lane == 0) {
+          const uint32_t sf_bytes = ((sfa_copy ? 1 : 0) + sfb_copies) * nk64 * kSfAtomBytes;
+          mbar_arrive_expect_tx(&sf_ready[stage], sf_bytes);
+          if (sfa_copy)
+            bulk_g2s(sSfa, p.sfa + ((arow / 128) * k64_per_row + k64_0) * kSfAtomBytes,
+                     nk64 * kSfAtomBytes, &sf_ready[stage]);
+          for (int blk = 0; blk < sfb_copies; ++blk) {
+            const int64_t rb = n0 / 128 + blk;
+            bulk_g2s(sSfb + blk * kK64PerStage * kSfAtomBytes,
+                     p.sfb + (rb * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
+                     &sf_ready[stage]);
+          }
+          const uint32_t fullc = full0 + stage * 8;
+          mbar_arrive_expect_tx_cluster(fullc, C::kABytes + C::kBBytes);
+          tma_load_2d_pair(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(arow), fullc);
+          tma_load_2d_pair(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(brow), fullc);
+        }
+        __syncwarp();
+      }
+    }
+    if (ok) {
+      const uint32_t used = it < STAGES ? it : STAGES;
+      for (uint32_t i = 0; i < used; ++i) {
+        const uint32_t j = it - used + i;
+        if (!mbar_wait_cluster_warp(&empty[j % STAGES], (j / STAGES) & 1, kWaitTimeoutNs)) {
+          if (lane == 0) report_timeout(p.dev_status);
+          break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer (even CTA)
+    if (leader && lane == 0) {
+      uint32_t it = 0;
+      uint32_t tile_iter = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += npairs, ++tile_iter) {
+        if (tile_iter > 0 && !mbar_wait_cluster(acc_empty, (tile_iter - 1) & 1, kWaitTimeoutNs)) {
+          report_timeout(p.dev_status);
+          break;
+        }
+        tc_fence_after();
+        int prev = -1;  // stage whose release is still to be issued (see the single-CTA kernel)
+        for (int kt = 0; kt < num_kt; ++kt, ++it) {
+          const int stage = static_cast<int>(it % STAGES);
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait_cluster(&full[stage], round & 1, kWaitTimeoutNs) ||
+              !mbar_wait_cluster(&sf_full[stage], round & 1, kWaitTimeoutNs)) {
+            report_timeout(p.dev_status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (prev >= 0) tc_commit_pair(&empty[prev], 0x3);
+          const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
+          const uint32_t sA = smem_u32(smem + C::kOffA + stage * C::kABytes);
+          const uint32_t sB = smem_u32(smem + C::kOffB + stage * C::kBBytes);
+          const uint32_t slot = tmem_base + C::kSfCol0 + stage * C::kSlotCols;
+          for (int a = 0; a < nk64; ++a) {
+            mma_nvf4_pair(tmem_base, desc_sw128(sA + a * 32), desc_sw128(sB + a * 32), C::kIdesc,
+                          slot + a * C::kSfaColsPerK64,
+                          slot + kK64PerStage * C::kSfaColsPerK64 + a * C::kSfbColsPerK64,
+                          (kt | a) != 0 ? 1u : 0u);
+          }
+          prev = stage;
+        }
+        if (prev >= 0) tc_commit_pair(&empty[prev], 0x3);
+        if (ok) tc_commit_pair(acc_full, 0x3);
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kSfWarp0 && warp < kSfWarp0 + 4) {
+    // ------------------------------------------------------------------ scale warps (each CTA)
+    const int q = warp & 3;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t sf_full0 = mapa_shared(smem_u32(&sf_full[0]), 0);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = pair; t < num_tiles && ok; t += npairs) {
+      for (int kt = 0; kt < num_kt; ++kt, ++it) {
+        const int stage = static_cast<int>(it % STAGES);
+        const uint32_t round = it / STAGES;
+        if (!mbar_wait_warp(&sf_ready[stage], round & 1, kWaitTimeoutNs)) {
+          if (lane == 0) report_timeout(p.dev_status);
+          ok = false;
+          break;
+        }
+        const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
+        const uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
+        const uint8_t *sSfb = smem + C::kOffSfb + stage * C::kSfbBytes;
+        const uint32_t slot = lane_base + C::kSfCol0 + stage * C::kSlotCols;
+        const uint32_t slot_b = slot + kK64PerStage * C::kSfaColsPerK64;
+        // same tensor-memory scale layout as the single-CTA kernel with a 256-row B operand
+        for (int a = 0; a < nk64; ++a) {
+          const uint32_t wa =
+              *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
+          tmem_st_x4_rep(slot + a * C::kSfaColsPerK64, wa);
+          const uint4 b0 = *reinterpret_cast<const uint4 *>(sSfb + a * kSfAtomBytes + lane * 16);
+          const uint4 b1 = *reinterpret_cast<const uint4 *>(
+              sSfb + (kK64PerStage + a) * kSfAtomBytes + lane * 16);
+          tmem_st_x8(slot_b + a * C::kSfbColsPerK64, b0, b1);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(sf_full0 + stage * 8);
+      }
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------------------------ epilogue (each CTA)
+    const int e = warp - kEpiWarp0;
+    const int q = warp & 3;
+    const int col0 = (e / 4) * C::kColsPerEpiWarp;
+    const int row = q * 32 + lane;
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(p.ga[0], p.gw[0]));
+    const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
+    uint32_t tile_iter = 0;
+    for (int t = pair; t < num_tiles; t += npairs, ++tile_iter) {
+      int64_t m0, n0;
+      tile_origin(t, m0, n0);
+      if (!mbar_wait_cluster_warp(acc_full, tile_iter & 1, kWaitTimeoutNs)) {
+        if (lane == 0) report_timeout(p.dev_status);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col0;
+      uint32_t h2[C::kColsPerEpiWarp / 2];
+#pragma unroll
+      for (int c = 0; c < C::kColsPerEpiWarp; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_acc + c, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          __half2 h = __floats2half2_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
+                                        __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
+          h2[c / 2 + j] = *reinterpret_cast<uint32_t *>(&h);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0);
+      const int64_t m = m0 + C::kHalf * rank + row;
+      if (m < p.M) {
+        __half *dst = p.out + m * p.N + n0 + col0;
+#pragma unroll
+        for (int j = 0; j < C::kColsPerEpiWarp / 8; ++j) {
+          if (n0 + col0 + 8 * j + 8 <= p.N) {
+            uint4 pk;
+            pk.x = h2[4 * j + 0];
+            pk.y = h2[4 * j + 1];
+            pk.z = h2[4 * j + 2];
+            pk.w = h2[4 * j + 3];
+            *reinterpret_cast<uint4 *>(dst + 8 * j) = pk;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------------------ host side
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -528,9 +844,76 @@ static cudaError_t run(const GemmArgs &g, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// CTA pairs that can be resident at once (a pair needs two SMs of one GPC, so this can be
+// below half the SM count); the persistent grid never exceeds it. Queried once per device.
+template <int STAGES>
+static int resident_pairs() {
+  constexpr int kMaxDevices = 64;
+  static std::once_flag once[kMaxDevices];
+  static int pairs[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::call_once(once[dev], [dev]() {
+    using C = PairCfg<STAGES>;
+    pairs[dev] = 0;
+    if (cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<STAGES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(C::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<STAGES>, &cfg) == cudaSuccess)
+      pairs[dev] = n;
+  });
+  return pairs[dev];
+}
+
+template <int STAGES>
+static cudaError_t run_pair(const GemmArgs &g, int num_sms, cudaStream_t st) {
+  (void)num_sms;
+  using C = PairCfg<STAGES>;
+  CUtensorMap ma, mb;
+  KernelParams p{};
+  const int64_t kb = g.K / 2;
+  if (!make_operand_map(&ma, g.a_q, g.M, kb, C::kHalf)) return cudaErrorInvalidValue;
+  if (!make_operand_map(&mb, g.w_q, g.N, kb, C::kHalf)) return cudaErrorInvalidValue;
+  p.sfa = g.a_sf;
+  p.sfb = g.w_sf;
+  p.sfb_8x4 = 0;
+  p.sfa_rows_padded = (g.M + 127) / 128 * 128;
+  p.sfb_rows_padded = (g.N + 127) / 128 * 128;
+  p.ga = g.a_g;
+  p.gw = g.w_g;
+  p.out = static_cast<__half *>(g.out);
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.dev_status = g.dev_status;
+  p.tiles_a = static_cast<int>((g.M + 255) / 256);
+  p.tiles_b = static_cast<int>((g.N + C::kN - 1) / C::kN);
+  const int64_t tiles = static_cast<int64_t>(p.tiles_a) * p.tiles_b;
+  const int resident = resident_pairs<STAGES>();
+  if (resident <= 0) return cudaErrorLaunchOutOfResources;
+  const int64_t pairs = tiles < resident ? tiles : resident;
+  gemm_nvfp4_pair_kernel<STAGES><<<static_cast<int>(2 * pairs), C::kThreads, C::kSmemBytes, st>>>(
+      ma, mb, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs &g, int num_sms, cudaStream_t st) {
   if (g.M <= 32) return run<32, 6, true>(g, num_sms, st);
-  return run<256, 4, false>(g, num_sms, st);
+  if (g.M < 256 || num_sms < 2) return run<256, 4, false>(g, num_sms, st);
+  return run_pair<5>(g, num_sms, st);
 }
 
 }  // namespace nvfp4

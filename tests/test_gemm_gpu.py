@@ -52,8 +52,12 @@ def _run(nv, ops, a_layout):
     return out.cpu().view(torch.int16).numpy().view(np.uint16)
 
 
+# M <= 32: swap-AB tiles; 33..255: single-CTA 128 x 256 tiles; M >= 256: CTA-pair 256 x 256
+# tiles (ragged M, N and K tails, and more tiles than resident pairs so the accumulator is
+# reused).
 SMALL = [(1, 256, 512), (8, 256, 512), (16, 256, 512), (32, 512, 1024), (3, 136, 64),
-         (33, 256, 512), (128, 256, 256), (130, 520, 320), (256, 1024, 2048), (300, 264, 4096)]
+         (33, 256, 512), (128, 256, 256), (130, 520, 320), (256, 1024, 2048), (300, 264, 4096),
+         (520, 776, 320), (4096, 2560, 512)]
 
 
 @pytest.mark.parametrize("M,N,K", SMALL)
