@@ -199,7 +199,7 @@ def run_ours(args, rank, world, torch, dist):
 
         def step(i):
             nv.nvfp4_quantize(copies[i % 3], g, per_token=True, sf_layout=nv.SF_128x4, q=q, sf=sf)
-        launches_per_step = 1
+        launches_per_step, period = 1, 3
         workload_desc = {"workload": "per-token NVFP4 quantize", "shape": [M, K], "input": "bf16",
                          "dist": "N(0,1), 0.1% of entries x50", "scales": "E4M3 128x4",
                          "global_scale": "fp32 per token", "l2": "input rotated over 3 copies (352 MB > 126 MB L2)"}
@@ -217,7 +217,7 @@ def run_ours(args, rank, world, torch, dist):
 
         def step(i):
             nv.swiglu_nvfp4_quantize(copies[i % 2], gdev, sf_layout=nv.SF_128x4, q=q, sf=sf)
-        launches_per_step = 1
+        launches_per_step, period = 1, 2
         workload_desc = {"workload": "fused SwiGLU + NVFP4 quantize", "shape": [M, 2 * H],
                          "input": "bf16", "dist": "N(0,1)", "scales": "E4M3 128x4",
                          "global_scale": "fp32 per tensor", "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
@@ -249,10 +249,13 @@ def run_ours(args, rank, world, torch, dist):
         alg = algorithmic(wl, M=M, N=N, K=K, a_layout=args.a_layout)
         kernel_key, kernel_name = f"gemm_{wl}", "gemm_nvfp4_kernel"
 
+        ws_bytes = nv.nvfp4_gemm_workspace_bytes(M, N, K)
+        gemm_ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+
         def step(i):
             aq, asf, wq, wsf = ops[i % ncopy]
-            nv.nvfp4_gemm(aq, asf, ga, wq, wsf, gw, a_layout=layout_code, out=out)
-        launches_per_step = 1
+            nv.nvfp4_gemm(aq, asf, ga, wq, wsf, gw, a_layout=layout_code, out=out, workspace=gemm_ws)
+        launches_per_step, period = 1, ncopy
         workload_desc = {"workload": f"NVFP4 GEMM ({wl})", "M": M, "N": N, "K": K,
                          "a_scales": args.a_layout, "w_scales": "128x4", "out": "fp16",
                          "l2": f"operands rotated over {ncopy} copies"}
@@ -267,6 +270,25 @@ def run_ours(args, rank, world, torch, dist):
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
+
+    # One CUDA graph per input copy, each holding one step (the library calls are made while
+    # the stream is captured: same kernels, same arguments). Replaying them keeps host launch
+    # cost out of the device timing, which matters for the tens-of-microsecond kernels.
+    run_step = step
+    if not args.no_graph:
+        graphs = []
+        for j in range(period):
+            gph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gph):
+                step(j)
+            graphs.append(gph)
+        torch.cuda.synchronize()
+
+        def run_step(i):
+            graphs[i % period].replay()
+        for i in range(args.warmup):
+            run_step(i)
+        torch.cuda.synchronize()
 
     # ---- timed region: K steps between two events on the launching stream. The step is one
     # launch of the path's kernel, so the kernel's average launch duration is the region's
@@ -285,7 +307,7 @@ def run_ours(args, rank, world, torch, dist):
     with Clocks(bus if rank == 0 else None) as clk:
         t0.record(stream)
         for i in range(args.steps):
-            step(args.warmup + i)
+            run_step(args.warmup + i)
         t1.record(stream)
         torch.cuda.synchronize()
     if dist is not None:
@@ -394,7 +416,8 @@ def run_ours(args, rank, world, torch, dist):
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {**workload_desc, "parallelism": f"replicas x{world}"},
+        "config": {**workload_desc, "parallelism": f"replicas x{world}",
+                   "timing": "direct calls" if args.no_graph else "CUDA-graph replay of each step's library call"},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary() if rank == 0 else None,
     }
@@ -510,6 +533,8 @@ def main():
     ap.add_argument("--a-layout", default="128x4", choices=["128x4", "8x4"])
     ap.add_argument("--cpu-rows", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time direct library calls instead of CUDA-graph replays of them")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -174,8 +174,13 @@ NVFP4_API int nvfp4_sf_unswizzle(const uint8_t *in, uint8_t *lin, int64_t R, int
                        void *stream);
 
 /*
- * Workspace bytes nvfp4_gemm needs for this shape (0 for every shape this build runs:
- * no split-K partials). Host only.
+ * Workspace bytes nvfp4_gemm needs for this shape on the current device. Non-zero only for
+ * M <= 32 (K <= 24576): that path splits the K range of the weight tiles evenly over the
+ * SMs ("stream-K") and keeps fp32 partial tiles [tiles][pieces][128][32] plus one int
+ * arrival counter per 128-row weight tile there (about 7.4 MB for N = 28672, K = 8192 on
+ * 148 SMs). The contents need no initialisation and are scratch after the call; calls that
+ * share a workspace must not overlap on the GPU. Returns 0 when no device is current.
+ * Host only.
  */
 NVFP4_API size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -193,7 +198,10 @@ NVFP4_API size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * a_g      device, one fp32 (the activation's encode scale).
  * w_q      device, [N, K/2] packed E2M1.   w_sf device, 128x4 layout.   w_g device fp32.
  * out      device, [M, N] fp16, row-major, row stride N.
- * workspace/workspace_bytes: >= nvfp4_gemm_workspace_bytes(M, N, K); may be NULL when 0.
+ * workspace/workspace_bytes: device, 16-byte aligned, >= nvfp4_gemm_workspace_bytes(M, N,
+ *          K) (NVFP4_ERR_INVALID_ARG when smaller); may be NULL when that is 0. The call
+ *          resets the counters it uses with an asynchronous memset on `stream` before the
+ *          kernel.
  * dev_status: device int32 or NULL. Each bounded wait inside the kernel that gives up
  *          (about 2 s without progress) ORs 1 into it and the kernel returns without
  *          finishing; the caller reads it after synchronizing (NVFP4_ERR_TIMEOUT).

@@ -459,6 +459,396 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------ small M
+
+// Small-M (decode) form, M <= 32: the operands swap roles (128 weight rows are the MMA's A
+// operand, the <= 32 tokens its N = 32 columns) and the work is split evenly over a resident
+// grid by K-steps ("stream-K"): the tiles x K-steps units are cut into one contiguous range
+// per CTA, so every CTA streams the same amount of weight bytes whatever the tile count.
+// A CTA whose range covers only part of a tile's K writes its fp32 partial accumulator to
+// the workspace; the last CTA to finish a tile (a per-tile arrival counter) adds the pieces
+// in piece order (deterministic) and writes the fp16 result. Activation scales: with the
+// 8x4 layout the <= 32 rows of all K (K/16 bytes each, four contiguous 8-row blocks) are
+// copied into shared memory once per CTA; with the 128x4 layout the activation atoms of
+// each ring stage are copied with the weight atoms.
+constexpr int kDecBN = 32;
+constexpr int kDecMaxSfbBytes = 48 * 1024;  // preloaded activation scales: K <= 24576
+
+template <int STAGES>
+struct DecCfg {
+  static constexpr int kABytes = kBM * kBKBytes;                 // 16 KB of weights
+  static constexpr int kBBytes = kDecBN * kBKBytes;              // 4 KB of activations
+  static constexpr int kSfaBytes = kK64PerStage * kSfAtomBytes;  // 2 KB of weight scales
+  static constexpr int kSfbBytes = kK64PerStage * kSfAtomBytes;  // 2 KB of activation atoms
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + STAGES * kABytes;
+  static constexpr int kOffSfa = kOffB + STAGES * kBBytes;
+  static constexpr int kOffSfbStage = kOffSfa + STAGES * kSfaBytes;
+  static constexpr int kOffBar = kOffSfbStage + STAGES * kSfbBytes;
+  static constexpr int kAccBufs = 2;
+  // full[S], empty[S], sf_full[S], acc_full[2], acc_empty[2], sfb_ready, tmem slot + flag
+  static constexpr int kBarBytes = (3 * STAGES + 2 * kAccBufs + 1) * 8 + 16;
+  static constexpr int kOffSfb = (kOffBar + kBarBytes + 127) / 128 * 128;  // 8x4 rows 0..31
+  static constexpr int kAccCols = kDecBN;
+  static constexpr int kSlotCols = kK64PerStage * (4 + 4);  // A scales 4 columns, B 4 (1 used)
+  static constexpr int kSfCol0 = kAccBufs * kAccCols;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kEpiWarps = 4;
+  static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
+  static_assert(kSfCol0 + STAGES * kSlotCols <= kTmemCols, "TMEM columns");
+  // the 8x4 copy holds 4 blocks of K/64 x 32 bytes
+  static constexpr int smem_bytes(int k64_total, bool sfb_8x4) {
+    return kOffSfb + (sfb_8x4 ? k64_total * 128 : 0) + 1024;
+  }
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(kDecBN >> 3) << 17) |
+                                     (uint32_t(kBM >> 4) << 24);
+};
+
+struct DecParams {
+  const uint8_t *w_sf;  // weight scales (128x4), MMA A operand
+  const uint8_t *a_sf;  // activation scales (128x4 or 8x4), MMA B operand
+  int a_sf_8x4;
+  int64_t a_sf_rows;    // rows of the activation-scale buffer (padded)
+  const float *ga;
+  const float *gw;
+  __half *out;
+  int64_t M, N, K;
+  int tiles;            // 128-row weight tiles
+  int max_pieces;       // CTAs a tile's K range can be split over
+  float *partials;      // [tiles][max_pieces][128][32] fp32
+  int *counters;        // [tiles], zero on entry
+  int32_t *dev_status;
+};
+
+// Contiguous unit range [u0, u1) of CTA c among G over U units (units = tile x K-step).
+__device__ __forceinline__ void dec_range(int64_t U, int c, int G, int64_t &u0, int64_t &u1) {
+  u0 = static_cast<int64_t>(c) * U / G;
+  u1 = static_cast<int64_t>(c + 1) * U / G;
+}
+
+// Index of the CTA whose range holds unit u.
+__device__ __forceinline__ int dec_owner(int64_t u, int G, int64_t U) {
+  return static_cast<int>(((u + 1) * G - 1) / U);
+}
+
+// AND of `v` over the `nthreads` threads of named barrier 1 (the epilogue warps).
+__device__ __forceinline__ bool epi_all(bool v, int nthreads) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, 1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
+    gemm_nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                             const __grid_constant__ CUtensorMap tmap_a, const DecParams p) {
+  using C = DecCfg<STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+  uint64_t *empty = full + STAGES;
+  uint64_t *sf_full = empty + STAGES;
+  uint64_t *acc_full = sf_full + STAGES;
+  uint64_t *acc_empty = acc_full + C::kAccBufs;
+  uint64_t *sfb_ready = acc_empty + C::kAccBufs;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sfb_ready + 1);
+  volatile int *last_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const uint8_t *sfb_8x4 = smem + C::kOffSfb;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_k64 = static_cast<int>(p.K / 64);
+  const int num_kt = (num_k64 + kK64PerStage - 1) / kK64PerStage;
+  const int64_t k64_per_row = p.K / 64;
+  const int64_t U = static_cast<int64_t>(p.tiles) * num_kt;
+  const int G = gridDim.x;
+  const int c = blockIdx.x;
+  int64_t u0, u1;
+  dec_range(U, c, G, u0, u1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 4);
+    }
+    for (int b = 0; b < C::kAccBufs; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], C::kEpiWarps);
+    }
+    mbar_init(sfb_ready, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tmap_w);
+    prefetch_tmap(&tmap_a);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (p.a_sf_8x4 && lane == 0) {
+      // rows 0..31 of the 8x4 activation scales: four blocks of K/64 x 32 contiguous bytes
+      const uint32_t blk = static_cast<uint32_t>(k64_per_row * 32);
+      const int nblk = static_cast<int>(p.a_sf_rows / 8);
+      mbar_arrive_expect_tx(sfb_ready, blk * nblk);
+      for (int b = 0; b < nblk; ++b)
+        bulk_g2s(smem + C::kOffSfb + b * blk, p.a_sf + static_cast<int64_t>(b) * blk, blk, sfb_ready);
+    }
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t u = u0; u < u1 && ok;) {
+      const int tile = static_cast<int>(u / num_kt);
+      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
+      const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
+      const int64_t w0 = static_cast<int64_t>(tile) * kBM;
+      for (int kt = kb; kt < ke; ++kt, ++it) {
+        const int stage = static_cast<int>(it % STAGES);
+        const uint32_t round = it / STAGES;
+        if (it >= STAGES && !mbar_wait_warp(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
+          if (lane == 0) report_timeout(p.dev_status);
+          ok = false;
+          break;
+        }
+        const int k64_0 = kt * kK64PerStage;
+        const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+        if (lane == 0) {
+          const uint32_t sf_bytes = (p.a_sf_8x4 ? 1 : 2) * nk64 * kSfAtomBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + sf_bytes);
+          tma_load_2d(smem + C::kOffA + stage * C::kABytes, &tmap_w, kt * kBKBytes,
+                      static_cast<int32_t>(w0), &full[stage]);
+          tma_load_2d(smem + C::kOffB + stage * C::kBBytes, &tmap_a, kt * kBKBytes, 0, &full[stage]);
+          bulk_g2s(smem + C::kOffSfa + stage * C::kSfaBytes,
+                   p.w_sf + ((w0 / 128) * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
+                   &full[stage]);
+          if (!p.a_sf_8x4)  // tokens 0..31 sit in the first 128-row block of the 128x4 scales
+            bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
+                     p.a_sf + static_cast<int64_t>(k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
+                     &full[stage]);
+        }
+        __syncwarp();
+      }
+      u += ke - kb;
+    }
+    if (ok) {
+      const uint32_t used = it < STAGES ? it : STAGES;
+      for (uint32_t i = 0; i < used; ++i) {
+        const uint32_t j = it - used + i;
+        if (!mbar_wait_warp(&empty[j % STAGES], (j / STAGES) & 1, kWaitTimeoutNs)) {
+          if (lane == 0) report_timeout(p.dev_status);
+          break;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, seg = 0;
+      bool ok = true;
+      for (int64_t u = u0; u < u1 && ok; ++seg) {
+        const int tile = static_cast<int>(u / num_kt);
+        const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
+        const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
+        const int buf = static_cast<int>(seg % C::kAccBufs);
+        const uint32_t use = seg / C::kAccBufs;
+        if (use > 0 && !mbar_wait_bounded(&acc_empty[buf], (use - 1) & 1, kWaitTimeoutNs)) {
+          report_timeout(p.dev_status);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + buf * C::kAccCols;
+        int prev = -1;
+        for (int kt = kb; kt < ke; ++kt, ++it) {
+          const int stage = static_cast<int>(it % STAGES);
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait_bounded(&full[stage], round & 1, kWaitTimeoutNs) ||
+              !mbar_wait_bounded(&sf_full[stage], round & 1, kWaitTimeoutNs)) {
+            report_timeout(p.dev_status);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (prev >= 0) tc_commit(&empty[prev]);
+          const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
+          const uint32_t sA = smem_u32(smem + C::kOffA + stage * C::kABytes);
+          const uint32_t sB = smem_u32(smem + C::kOffB + stage * C::kBBytes);
+          const uint32_t slot = tmem_base + C::kSfCol0 + stage * C::kSlotCols;
+          for (int a = 0; a < nk64; ++a) {
+            mma_nvf4(d_tmem, desc_sw128(sA + a * 32), desc_sw128(sB + a * 32), C::kIdesc, slot + a * 4,
+                     slot + kK64PerStage * 4 + a * 4, (kt != kb || a != 0) ? 1u : 0u);
+          }
+          prev = stage;
+        }
+        if (prev >= 0) tc_commit(&empty[prev]);
+        if (ok) tc_commit(&acc_full[buf]);
+        u += ke - kb;
+      }
+    }
+    __syncwarp();
+  } else if (warp >= kSfWarp0 && warp < kSfWarp0 + 4) {
+    // ------------------------------------------------------------------ scale warps
+    const int q = warp & 3;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t it = 0;
+    bool ok = true;
+    if (p.a_sf_8x4 && !mbar_wait_warp(sfb_ready, 0, kWaitTimeoutNs)) {
+      if (lane == 0) report_timeout(p.dev_status);
+      ok = false;
+    }
+    // token `lane`'s 8x4 words: block lane / 8, byte (lane % 8) * 4 of each 32-byte step
+    const uint8_t *my8x4 = sfb_8x4 + (lane / 8) * (k64_per_row * 32) + (lane % 8) * 4;
+    for (int64_t u = u0; u < u1 && ok;) {
+      const int tile = static_cast<int>(u / num_kt);
+      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
+      const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
+      for (int kt = kb; kt < ke; ++kt, ++it) {
+        const int stage = static_cast<int>(it % STAGES);
+        const uint32_t round = it / STAGES;
+        if (!mbar_wait_warp(&full[stage], round & 1, kWaitTimeoutNs)) {
+          if (lane == 0) report_timeout(p.dev_status);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int k64_0 = kt * kK64PerStage;
+        const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+        const uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
+        const uint32_t slot = lane_base + C::kSfCol0 + stage * C::kSlotCols;
+        // A (weights): row 32 q + lane's word at column (step base + q); B (tokens, N = 32):
+        // token lane's word at lane 32 q + lane, column (step base + 0), in every quarter.
+        for (int a = 0; a < nk64; ++a) {
+          const uint32_t wa =
+              *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
+          tmem_st_x4_rep(slot + a * 4, wa);
+          const uint32_t wb =
+              p.a_sf_8x4 ? *reinterpret_cast<const uint32_t *>(my8x4 + (k64_0 + a) * 32)
+                         : *reinterpret_cast<const uint32_t *>(
+                               smem + C::kOffSfbStage + stage * C::kSfbBytes + a * kSfAtomBytes + lane * 16);
+          tmem_st_x1(slot + kK64PerStage * 4 + a * 4, wb);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sf_full[stage]);
+      }
+      u += ke - kb;
+    }
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;  // weight row within the tile (accumulator lane)
+    const float alpha = __fdiv_rn(1.0f, __fmul_rn(p.ga[0], p.gw[0]));
+    uint32_t seg = 0;
+    for (int64_t u = u0; u < u1; ++seg) {
+      const int tile = static_cast<int>(u / num_kt);
+      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
+      const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
+      u += ke - kb;
+      const int buf = static_cast<int>(seg % C::kAccBufs);
+      const uint32_t use = seg / C::kAccBufs;
+      // the four epilogue warps leave together (they meet at named barriers below)
+      const bool got = mbar_wait_warp(&acc_full[buf], use & 1, kWaitTimeoutNs);
+      if (!epi_all(got, C::kEpiWarps * 32)) {
+        if (lane == 0) report_timeout(p.dev_status);
+        break;
+      }
+      tc_fence_after();
+      float vals[kDecBN];
+      const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
+#pragma unroll
+      for (int cc = 0; cc < kDecBN; cc += 8) {
+        uint32_t v[8];
+        tmem_ld_32x32b_x8(t_acc + cc, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) vals[cc + j] = __uint_as_float(v[j]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      const int64_t n = static_cast<int64_t>(tile) * kBM + row;
+      if (kb == 0 && ke == num_kt) {
+        if (n < p.N) {
+#pragma unroll
+          for (int j = 0; j < kDecBN; ++j)
+            if (j < p.M) p.out[j * p.N + n] = __float2half_rn(__fmul_rn(vals[j], alpha));
+        }
+        continue;
+      }
+      // partial tile: publish this piece, the last arriver sums the pieces in order
+      const int64_t tu0 = static_cast<int64_t>(tile) * num_kt;
+      const int first = dec_owner(tu0, G, U);
+      const int pieces = dec_owner(tu0 + num_kt - 1, G, U) - first + 1;
+      const int piece = c - first;
+      float *part_base = p.partials + static_cast<int64_t>(tile) * p.max_pieces * kBM * kDecBN;
+      float4 *mine = reinterpret_cast<float4 *>(part_base + (static_cast<int64_t>(piece) * kBM + row) * kDecBN);
+#pragma unroll
+      for (int j = 0; j < kDecBN / 4; ++j)
+        mine[j] = make_float4(vals[4 * j], vals[4 * j + 1], vals[4 * j + 2], vals[4 * j + 3]);
+      asm volatile("bar.sync 1, %0;" ::"n"(C::kEpiWarps * 32) : "memory");
+      if (warp == kEpiWarp0 && lane == 0) {
+        __threadfence();
+        const int old = atomicAdd(p.counters + tile, 1);
+        *last_flag = (old == pieces - 1) ? 1 : 0;
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(C::kEpiWarps * 32) : "memory");
+      const bool last = *last_flag != 0;
+      asm volatile("bar.sync 1, %0;" ::"n"(C::kEpiWarps * 32) : "memory");  // flag read before reuse
+      if (!last) continue;
+      __threadfence();
+      float acc[kDecBN];
+#pragma unroll
+      for (int j = 0; j < kDecBN; ++j) acc[j] = 0.0f;
+      for (int pc = 0; pc < pieces; ++pc) {
+        if (pc == piece) {
+#pragma unroll
+          for (int j = 0; j < kDecBN; ++j) acc[j] = __fadd_rn(acc[j], vals[j]);
+        } else {
+          const float4 *src = reinterpret_cast<const float4 *>(
+              part_base + (static_cast<int64_t>(pc) * kBM + row) * kDecBN);
+#pragma unroll
+          for (int j = 0; j < kDecBN / 4; ++j) {
+            const float4 v4 = __ldcg(src + j);
+            acc[4 * j] = __fadd_rn(acc[4 * j], v4.x);
+            acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], v4.y);
+            acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], v4.z);
+            acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], v4.w);
+          }
+        }
+      }
+      if (n < p.N) {
+#pragma unroll
+        for (int j = 0; j < kDecBN; ++j)
+          if (j < p.M) p.out[j * p.N + n] = __float2half_rn(__fmul_rn(acc[j], alpha));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------------------ CTA pairs
 
 // Large-M form: a cluster of two CTAs computes a 256 x 256 tile with the pair MMA
@@ -788,8 +1178,8 @@ static EncodeTiledFn encode_fn() {
 
 // 2-D map over a packed [rows, K/2] byte matrix, box = 128 bytes x box_rows, 128-byte swizzle;
 // reads past the last row or column are zero-filled.
-static bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t k_bytes,
-                             int box_rows) {
+static bool encode_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t k_bytes,
+                               int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k_bytes), static_cast<cuuint64_t>(rows)};
@@ -800,6 +1190,72 @@ static bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, i
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Encoding a tensor map is host work of about a microsecond; decode-sized GEMMs run in tens
+// of microseconds and are launched with the same operands over and over, so maps are kept
+// in a small table keyed by (address, rows, row bytes, box rows). The map holds no device
+// state: a hit for a freed-and-reused address describes the same layout and stays valid.
+struct MapKey {
+  const void *base;
+  int64_t rows, k_bytes;
+  int box_rows;
+};
+
+static bool make_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t k_bytes,
+                             int box_rows) {
+  constexpr int kSlots = 64;
+  static std::mutex mu;
+  static MapKey keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static int used = 0, next = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i) {
+      const MapKey &k = keys[i];
+      if (k.base == base && k.rows == rows && k.k_bytes == k_bytes && k.box_rows == box_rows) {
+        *map = maps[i];
+        return true;
+      }
+    }
+  }
+  if (!encode_operand_map(map, base, rows, k_bytes, box_rows)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  const int slot = used < kSlots ? used++ : next;
+  next = (slot + 1) % kSlots;
+  keys[slot] = MapKey{base, rows, k_bytes, box_rows};
+  maps[slot] = *map;
+  return true;
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel, device and size: the
+// call costs host time on every launch otherwise.
+template <typename Kernel>
+static cudaError_t ensure_smem_attr(Kernel kernel, int bytes) {
+  struct Entry {
+    const void *fn;
+    int dev;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry done[64];
+  static int n = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const void *fn = reinterpret_cast<const void *>(kernel);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (done[i].fn == fn && done[i].dev == dev && done[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < n; ++i)
+    if (done[i].fn == fn && done[i].dev == dev) {
+      done[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (n < 64) done[n++] = Entry{fn, dev, bytes};
+  return cudaSuccess;
 }
 
 template <int BN, int STAGES, bool SWAP>
@@ -837,8 +1293,7 @@ static cudaError_t run(const GemmArgs &g, int num_sms, cudaStream_t st) {
   p.tiles_b = static_cast<int>((rows_b + BN - 1) / BN);
   const int64_t tiles = static_cast<int64_t>(p.tiles_a) * p.tiles_b;
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel<BN, STAGES, SWAP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  cudaError_t e = ensure_smem_attr(gemm_nvfp4_kernel<BN, STAGES, SWAP>, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   gemm_nvfp4_kernel<BN, STAGES, SWAP><<<grid, C::kThreads, C::kSmemBytes, st>>>(ma, mb, p);
   return cudaGetLastError();
@@ -856,10 +1311,7 @@ static int resident_pairs() {
   std::call_once(once[dev], [dev]() {
     using C = PairCfg<STAGES>;
     pairs[dev] = 0;
-    if (cudaFuncSetAttribute(gemm_nvfp4_pair_kernel<STAGES>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return;
+    if (ensure_smem_attr(gemm_nvfp4_pair_kernel<STAGES>, C::kSmemBytes) != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(C::kThreads, 1, 1);
@@ -910,8 +1362,77 @@ static cudaError_t run_pair(const GemmArgs &g, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// Small-M stream-K layout for a device with num_sms SMs: grid, pieces per tile, workspace.
+struct DecPlan {
+  int grid = 0;
+  int tiles = 0;
+  int max_pieces = 0;
+  size_t partial_bytes = 0;
+  size_t counter_bytes = 0;
+  bool usable = false;
+};
+
+static DecPlan dec_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+  DecPlan d;
+  if (M > kDecBN || K / 64 * 128 > kDecMaxSfbBytes) return d;
+  const int64_t num_kt = (K / 64 + kK64PerStage - 1) / kK64PerStage;
+  d.tiles = static_cast<int>((N + kBM - 1) / kBM);
+  const int64_t U = d.tiles * num_kt;
+  d.grid = static_cast<int>(U < num_sms ? U : num_sms);
+  if (d.grid < 1) return d;
+  const int64_t umin = U / d.grid;  // every CTA holds at least this many units
+  int64_t mp = (num_kt - 1 + umin - 1) / umin + 1;
+  if (mp > num_kt) mp = num_kt;
+  d.max_pieces = static_cast<int>(mp);
+  d.partial_bytes = static_cast<size_t>(d.tiles) * d.max_pieces * kBM * kDecBN * sizeof(float);
+  d.counter_bytes = (static_cast<size_t>(d.tiles) * sizeof(int) + 255) / 256 * 256;
+  d.usable = true;
+  return d;
+}
+
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  const DecPlan d = dec_plan(M, N, K, num_sms);
+  return d.usable ? d.partial_bytes + d.counter_bytes : 0;
+}
+
+template <int STAGES>
+static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t st) {
+  using C = DecCfg<STAGES>;
+  CUtensorMap mw, ma;
+  const int64_t kb = g.K / 2;
+  if (!make_operand_map(&mw, g.w_q, g.N, kb, kBM)) return cudaErrorInvalidValue;
+  if (!make_operand_map(&ma, g.a_q, g.M, kb, kDecBN)) return cudaErrorInvalidValue;
+  DecParams p{};
+  p.w_sf = g.w_sf;
+  p.a_sf = g.a_sf;
+  p.a_sf_8x4 = g.a_layout == kSf8x4 ? 1 : 0;
+  p.a_sf_rows = p.a_sf_8x4 ? (g.M + 7) / 8 * 8 : (g.M + 127) / 128 * 128;
+  p.ga = g.a_g;
+  p.gw = g.w_g;
+  p.out = static_cast<__half *>(g.out);
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.tiles = d.tiles;
+  p.max_pieces = d.max_pieces;
+  p.partials = static_cast<float *>(g.workspace);
+  p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(g.workspace) + d.partial_bytes);
+  p.dev_status = g.dev_status;
+  cudaError_t e = cudaMemsetAsync(p.counters, 0, d.counter_bytes, st);
+  if (e != cudaSuccess) return e;
+  const int smem = C::smem_bytes(static_cast<int>(g.K / 64), p.a_sf_8x4 != 0);
+  e = ensure_smem_attr(gemm_nvfp4_decode_kernel<STAGES>, smem);
+  if (e != cudaSuccess) return e;
+  gemm_nvfp4_decode_kernel<STAGES><<<d.grid, C::kThreads, smem, st>>>(mw, ma, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs &g, int num_sms, cudaStream_t st) {
-  if (g.M <= 32) return run<32, 6, true>(g, num_sms, st);
+  if (g.M <= 32) {
+    const DecPlan d = dec_plan(g.M, g.N, g.K, num_sms);
+    if (d.usable) return run_decode<7>(g, d, st);
+    return run<32, 6, true>(g, num_sms, st);
+  }
   if (g.M < 256 || num_sms < 2) return run<256, 4, false>(g, num_sms, st);
   return run_pair<5>(g, num_sms, st);
 }

@@ -44,7 +44,12 @@ struct GemmArgs {
   void *out;
   int64_t M, N, K;
   int32_t *dev_status;
+  void *workspace;
+  size_t workspace_bytes;
 };
 cudaError_t launch_gemm(const GemmArgs &args, int num_sms, cudaStream_t st);
+// Workspace the GEMM needs for (M, N, K) on a device with num_sms SMs (split-K partial sums
+// and tile counters of the small-M path; 0 otherwise).
+size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
 
 }  // namespace nvfp4

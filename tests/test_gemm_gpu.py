@@ -57,7 +57,8 @@ def _run(nv, ops, a_layout):
 # reused).
 SMALL = [(1, 256, 512), (8, 256, 512), (16, 256, 512), (32, 512, 1024), (3, 136, 64),
          (33, 256, 512), (128, 256, 256), (130, 520, 320), (256, 1024, 2048), (300, 264, 4096),
-         (520, 776, 320), (4096, 2560, 512)]
+         (520, 776, 320), (4096, 2560, 512),
+         (2, 20480, 1024), (32, 4096, 3072), (17, 1032, 8192)]
 
 
 @pytest.mark.parametrize("M,N,K", SMALL)
@@ -69,6 +70,26 @@ def test_gemm_parity_small(M, N, K):
     for layout in layouts:
         got = _run(nv, ops, layout)
         gemm_close(got, ref)
+
+
+def test_gemm_small_m_workspace_contract():
+    """M <= 32 needs the split-K workspace; a smaller one is refused before any launch."""
+    nv = require_cuda()
+    import ctypes
+    L = nv.lib()
+    M, N, K = 8, 28672, 8192
+    need = L.nvfp4_gemm_workspace_bytes(M, N, K)
+    assert need >= (N // 128) * 128 * 32 * 4
+    assert L.nvfp4_gemm_workspace_bytes(33, N, K) == 0
+    ops = _random_operands(M, 256, 512, seed=5)
+    dev = _to_device(nv, *ops, orc.L128x4)
+    out = torch.empty(M, 256, dtype=torch.float16, device="cuda")
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    rc = L.nvfp4_gemm(p(dev["a_q"]), p(dev["a_sf"]), orc.L128x4, p(dev["a_g"]), p(dev["w_q"]),
+                      p(dev["w_sf"]), p(dev["w_g"]), p(out), M, 256, 512, p(small), 16, None,
+                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == nv.ERR_INVALID_ARG
 
 
 def test_gemm_tiny_workload():
