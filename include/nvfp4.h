@@ -4,7 +4,9 @@
  *
  * Conventions (all entry points):
  *  - Every pointer argument named as "device" is caller-owned device memory; the library
- *    never allocates, frees or retains it. Sizes are element counts unless stated.
+ *    never allocates, frees or retains it (scratch comes from caller workspaces, or from
+ *    the fixed library array of nvfp4_global_scale_noalloc). Sizes are element counts
+ *    unless stated.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Calls
  *    are asynchronous on that stream and return once the work is enqueued.
  *  - Return value: an nvfp4_status. Argument errors are detected on the host before any
@@ -13,10 +15,12 @@
  *    stream as CUDA errors; a bounded wait that gave up inside the GEMM is reported through
  *    its `dev_status` word.
  *  - Functions are thread-safe and keep no per-call state: the same call may run on
- *    different streams concurrently. The first call on a device resolves the tensor-map
- *    encoder and the SM count once; later calls issue no device queries.
- *  - No entry point is a no-op on empty input: M == 0 (or N == 0) is accepted and enqueues
- *    nothing; K, H must be positive.
+ *    different streams concurrently (calls sharing a workspace must not overlap). The first
+ *    call on a device resolves the tensor-map encoder, the SM count and the GEMM's
+ *    resident cluster count once; encoded tensor maps are cached on the host; later calls
+ *    issue no device queries.
+ *  - Empty input is valid: M == 0 (or N == 0) returns NVFP4_OK and enqueues nothing. K and
+ *    H must be positive.
  *
  * Number formats: E2M1 (OCP MX FP4: magnitudes {0, 0.5, 1, 1.5, 2, 3, 4, 6}, sign bit 3),
  * packed two per byte, element 2j in the low nibble of byte j. Block scales are E4M3
