@@ -217,6 +217,22 @@ NVFP4_API int nvfp4_gemm(const uint8_t *a_q, const uint8_t *a_sf, int a_layout, 
                int64_t N, int64_t K, void *workspace, size_t workspace_bytes, int32_t *dev_status,
                void *stream);
 
+/*
+ * The GEMM for an activation quantized per token (nvfp4_quantize with per_token = 1): same
+ * arguments and contract as nvfp4_gemm except that a_g is a device fp32 [M] array, one
+ * encode scale per activation row, so
+ *   out[m,n] = fp16( sum_k E2M1(a[m,k]) * E4M3(sa[m,k/16]) * E2M1(w[n,k]) * E4M3(sw[n,k/16])
+ *                    / (a_g[m] * w_g) ).
+ * It closes the loop the per-token quantize PR ("perf: optimize per-token nvfp4 quantization
+ * kernel", FlashInfer PR #3237, which tests per-token scales in the MoE path) implies: the
+ * row scale is applied in the epilogue, fp32(1 / (a_g[m] * w_g)) times the fp32 accumulator.
+ */
+NVFP4_API int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int a_layout,
+                                   const float *a_g, const uint8_t *w_q, const uint8_t *w_sf,
+                                   const float *w_g, void *out, int64_t M, int64_t N, int64_t K,
+                                   void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                                   void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -38,6 +38,8 @@ SIGNATURES = {
     "nvfp4_gemm_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz,
                           _vp, _vp]),
+    "nvfp4_gemm_per_token": (_i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
+                                    _vp, _sz, _vp, _vp]),
 }
 
 _lib = None
@@ -200,8 +202,13 @@ def nvfp4_sf_unswizzle(buf: torch.Tensor, R: int, C: int, layout: int = SF_128x4
 def nvfp4_gemm(a_q: torch.Tensor, a_sf: torch.Tensor, a_g: torch.Tensor, w_q: torch.Tensor,
                w_sf: torch.Tensor, w_g: torch.Tensor, a_layout: int = SF_128x4,
                out: torch.Tensor | None = None, dev_status: torch.Tensor | None = None,
-               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """out[M, N] fp16 = dequant(a_q) @ dequant(w_q)^T (K = 2 * a_q.shape[1])."""
+               workspace: torch.Tensor | None = None, per_token_a: bool = False,
+               stream=None) -> torch.Tensor:
+    """out[M, N] fp16 = dequant(a_q) @ dequant(w_q)^T (K = 2 * a_q.shape[1]).
+
+    per_token_a: a_g is fp32 [M], one encode scale per activation row (the g that
+    nvfp4_quantize(per_token=True) writes); otherwise a_g is fp32 [1].
+    """
     M, K2 = a_q.shape
     N = w_q.shape[0]
     K = 2 * K2
@@ -210,8 +217,11 @@ def nvfp4_gemm(a_q: torch.Tensor, a_sf: torch.Tensor, a_g: torch.Tensor, w_q: to
     nbytes = nvfp4_gemm_workspace_bytes(M, N, K)
     if workspace is None and nbytes > 0:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=a_q.device)
-    _check(lib().nvfp4_gemm(_ptr(a_q), _ptr(a_sf), a_layout, _ptr(a_g), _ptr(w_q), _ptr(w_sf),
-                            _ptr(w_g), _ptr(out), M, N, K, _ptr(workspace),
-                            0 if workspace is None else workspace.numel(), _ptr(dev_status),
-                            _stream(stream)), "nvfp4_gemm")
+    if per_token_a and a_g.numel() != M:
+        raise ValueError(f"per_token_a needs a_g with M = {M} elements, got {a_g.numel()}")
+    fn = lib().nvfp4_gemm_per_token if per_token_a else lib().nvfp4_gemm
+    _check(fn(_ptr(a_q), _ptr(a_sf), a_layout, _ptr(a_g), _ptr(w_q), _ptr(w_sf), _ptr(w_g),
+              _ptr(out), M, N, K, _ptr(workspace), 0 if workspace is None else workspace.numel(),
+              _ptr(dev_status), _stream(stream)),
+           "nvfp4_gemm_per_token" if per_token_a else "nvfp4_gemm")
     return out

@@ -181,10 +181,10 @@ size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return gemm_workspace_bytes(M, N, K, d->num_sms);
 }
 
-int nvfp4_gemm(const uint8_t *a_q, const uint8_t *a_sf, int a_layout, const float *a_g,
-               const uint8_t *w_q, const uint8_t *w_sf, const float *w_g, void *out, int64_t M,
-               int64_t N, int64_t K, void *workspace, size_t workspace_bytes, int32_t *dev_status,
-               void *stream) {
+static int gemm_impl(const uint8_t *a_q, const uint8_t *a_sf, int a_layout, const float *a_g,
+                     int a_g_per_row, const uint8_t *w_q, const uint8_t *w_sf, const float *w_g,
+                     void *out, int64_t M, int64_t N, int64_t K, void *workspace,
+                     size_t workspace_bytes, int32_t *dev_status, void *stream) {
   if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_INVALID_ARG;
   if (a_layout != NVFP4_SF_128x4 && a_layout != NVFP4_SF_8x4) return NVFP4_ERR_INVALID_ARG;
   if (a_layout == NVFP4_SF_8x4 && M > 32) return NVFP4_ERR_UNSUPPORTED;
@@ -204,9 +204,26 @@ int nvfp4_gemm(const uint8_t *a_q, const uint8_t *a_sf, int a_layout, const floa
   const size_t ws_need = gemm_workspace_bytes(M, N, K, d->num_sms);
   if (ws_need > 0 && (workspace == nullptr || workspace_bytes < ws_need)) return NVFP4_ERR_INVALID_ARG;
   if (ws_need > 0 && !aligned16(workspace)) return NVFP4_ERR_MISALIGNED;
-  GemmArgs g{a_q, a_sf, a_layout, a_g, w_q, w_sf, w_g, out, M, N, K, dev_status, workspace,
-             workspace_bytes};
+  GemmArgs g{a_q,    a_sf,      a_layout,        a_g,        w_q,      w_sf,
+             w_g,    out,       M,               N,          K,        dev_status,
+             workspace, workspace_bytes, a_g_per_row};
   return finish(launch_gemm(g, d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_gemm(const uint8_t *a_q, const uint8_t *a_sf, int a_layout, const float *a_g,
+               const uint8_t *w_q, const uint8_t *w_sf, const float *w_g, void *out, int64_t M,
+               int64_t N, int64_t K, void *workspace, size_t workspace_bytes, int32_t *dev_status,
+               void *stream) {
+  return gemm_impl(a_q, a_sf, a_layout, a_g, 0, w_q, w_sf, w_g, out, M, N, K, workspace,
+                   workspace_bytes, dev_status, stream);
+}
+
+int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int a_layout, const float *a_g,
+                         const uint8_t *w_q, const uint8_t *w_sf, const float *w_g, void *out,
+                         int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                         int32_t *dev_status, void *stream) {
+  return gemm_impl(a_q, a_sf, a_layout, a_g, 1, w_q, w_sf, w_g, out, M, N, K, workspace,
+                   workspace_bytes, dev_status, stream);
 }
 
 }  // extern "C"

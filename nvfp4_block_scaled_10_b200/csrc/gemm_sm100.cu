@@ -140,12 +140,21 @@ struct KernelParams {
   int64_t sfa_rows_padded;  // rows of the A-scale buffer
   const float *ga;
   const float *gw;
+  int ga_per_row;   // ga holds one encode scale per activation row (per-token quantization)
   __half *out;
   int64_t M, N, K;  // problem shape in the caller's (unswapped) terms
   int tiles_a;      // tiles along the MMA A operand (128 rows each)
   int tiles_b;      // tiles along the MMA B operand (BN rows each)
   int32_t *dev_status;
 };
+
+// Output scale 1 / (ga * gw) of activation row m: ga[m] when the activation was quantized
+// with one encode scale per row, else the scalar ga[0].
+__device__ __forceinline__ float out_alpha(const float *ga, int per_row, const float *gw, int64_t m,
+                                           int64_t M) {
+  const float a = per_row ? (m < M ? ga[m] : 1.0f) : ga[0];
+  return __fdiv_rn(1.0f, __fmul_rn(a, gw[0]));
+}
 
 __device__ __forceinline__ void report_timeout(int32_t *dev_status) {
   if (dev_status != nullptr) atomicOr(dev_status, kDevErrTimeout);
@@ -378,11 +387,12 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int col0 = (e / 4) * C::kColsPerEpiWarp;
     const int row = q * 32 + lane;
-    const float alpha = __fdiv_rn(1.0f, __fmul_rn(p.ga[0], p.gw[0]));
     uint32_t tile_iter = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tile_iter) {
       int64_t a0, b0;
       tile_origin(t, a0, b0);
+      // this thread's output row (unswapped), or per column below (swapped)
+      const float alpha = out_alpha(p.ga, p.ga_per_row, p.gw, a0 + row, p.M);
       const int buf = static_cast<int>(tile_iter % C::kAccBufs);
       const uint32_t use = tile_iter / C::kAccBufs;
       if (!mbar_wait_warp(&acc_full[buf], use & 1, kWaitTimeoutNs)) {
@@ -434,7 +444,9 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
           tmem_ld_32x32b_x8(t_acc + c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) vals[c + j] = __fmul_rn(__uint_as_float(v[j]), alpha);
+          for (int j = 0; j < 8; ++j)
+            vals[c + j] = __fmul_rn(__uint_as_float(v[j]),
+                                    out_alpha(p.ga, p.ga_per_row, p.gw, b0 + col0 + c + j, p.M));
         }
         tc_fence_before();
         __syncwarp();
@@ -511,6 +523,7 @@ struct DecParams {
   int64_t a_sf_rows;    // rows of the activation-scale buffer (padded)
   const float *ga;
   const float *gw;
+  int ga_per_row;       // ga holds one encode scale per token
   __half *out;
   int64_t M, N, K;
   int tiles;            // 128-row weight tiles
@@ -754,7 +767,9 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;  // weight row within the tile (accumulator lane)
-    const float alpha = __fdiv_rn(1.0f, __fmul_rn(p.ga[0], p.gw[0]));
+    float alpha[kDecBN];  // per token (accumulator column)
+#pragma unroll
+    for (int j = 0; j < kDecBN; ++j) alpha[j] = out_alpha(p.ga, p.ga_per_row, p.gw, j, p.M);
     uint32_t seg = 0;
     for (int64_t u = u0; u < u1; ++seg) {
       const int tile = static_cast<int>(u / num_kt);
@@ -788,7 +803,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
         if (n < p.N) {
 #pragma unroll
           for (int j = 0; j < kDecBN; ++j)
-            if (j < p.M) p.out[j * p.N + n] = __float2half_rn(__fmul_rn(vals[j], alpha));
+            if (j < p.M) p.out[j * p.N + n] = __float2half_rn(__fmul_rn(vals[j], alpha[j]));
         }
         continue;
       }
@@ -836,7 +851,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
       if (n < p.N) {
 #pragma unroll
         for (int j = 0; j < kDecBN; ++j)
-          if (j < p.M) p.out[j * p.N + n] = __float2half_rn(__fmul_rn(acc[j], alpha));
+          if (j < p.M) p.out[j * p.N + n] = __float2half_rn(__fmul_rn(acc[j], alpha[j]));
       }
     }
   }
@@ -1102,12 +1117,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
     const int q = warp & 3;
     const int col0 = (e / 4) * C::kColsPerEpiWarp;
     const int row = q * 32 + lane;
-    const float alpha = __fdiv_rn(1.0f, __fmul_rn(p.ga[0], p.gw[0]));
     const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
     uint32_t tile_iter = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++tile_iter) {
       int64_t m0, n0;
       tile_origin(t, m0, n0);
+      const float alpha = out_alpha(p.ga, p.ga_per_row, p.gw, m0 + C::kHalf * rank + row, p.M);
       if (!mbar_wait_cluster_warp(acc_full, tile_iter & 1, kWaitTimeoutNs)) {
         if (lane == 0) report_timeout(p.dev_status);
         break;
@@ -1282,6 +1297,7 @@ static cudaError_t run(const GemmArgs &g, int num_sms, cudaStream_t st) {
   }
   p.ga = g.a_g;
   p.gw = g.w_g;
+  p.ga_per_row = g.a_g_per_row;
   p.out = static_cast<__half *>(g.out);
   p.M = g.M;
   p.N = g.N;
@@ -1346,6 +1362,7 @@ static cudaError_t run_pair(const GemmArgs &g, int num_sms, cudaStream_t st) {
   p.sfb_rows_padded = (g.N + 127) / 128 * 128;
   p.ga = g.a_g;
   p.gw = g.w_g;
+  p.ga_per_row = g.a_g_per_row;
   p.out = static_cast<__half *>(g.out);
   p.M = g.M;
   p.N = g.N;
@@ -1409,6 +1426,7 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   p.a_sf_rows = p.a_sf_8x4 ? (g.M + 7) / 8 * 8 : (g.M + 127) / 128 * 128;
   p.ga = g.a_g;
   p.gw = g.w_g;
+  p.ga_per_row = g.a_g_per_row;
   p.out = static_cast<__half *>(g.out);
   p.M = g.M;
   p.N = g.N;

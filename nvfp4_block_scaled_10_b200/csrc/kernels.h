@@ -46,6 +46,7 @@ struct GemmArgs {
   int32_t *dev_status;
   void *workspace;
   size_t workspace_bytes;
+  int a_g_per_row;  // a_g is [M]: one activation encode scale per row
 };
 cudaError_t launch_gemm(const GemmArgs &args, int num_sms, cudaStream_t st);
 // Workspace the GEMM needs for (M, N, K) on a device with num_sms SMs (split-K partial sums

@@ -78,6 +78,7 @@ def lib():
             "orc_sf_unswizzle": (None, [vp, i64, i64, i32, vp]),
             "orc_gemm": (None, [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, vp]),
             "orc_dequantize": (None, [vp, vp, f32, i64, i64, vp]),
+            "orc_dequantize_rows": (None, [vp, vp, vp, i64, i64, vp]),
             "orc_e2m1_encode_array": (None, [vp, i64, vp]),
             "orc_e4m3_encode_array": (None, [vp, i64, vp]),
             "orc_exp_array": (None, [vp, i64, vp]),
@@ -274,14 +275,32 @@ def dequantize(q, sf_lin, g) -> np.ndarray:
     return out
 
 
+def dequantize_rows(q, sf_lin, g_rows) -> np.ndarray:
+    """fp64 values E2M1(q) * E4M3(s) / g[r] of a packed operand [rows, K/2] quantized with
+    one encode scale per row."""
+    qq = _c(q, np.uint8)
+    ss = _c(sf_lin, np.uint8)
+    gg = _c(np.asarray(g_rows, dtype=np.float32).reshape(-1), np.float32)
+    rows, K2 = qq.shape
+    K = 2 * K2
+    assert ss.shape == (rows, K // 16) and gg.shape == (rows,)
+    out = np.zeros((rows, K), np.float64)
+    lib().orc_dequantize_rows(_p(qq), _p(ss), _p(gg), rows, K, _p(out))
+    return out
+
+
 def gemm(a_q, a_sf_lin, a_g, w_q, w_sf_lin, w_g, want_f64: bool = False):
     """D = fp16_rn(deq(A) @ deq(W)^T): dequantization in the C oracle, the fp64 product by
     numpy's matmul (a library step), one rounding to fp16 by the C oracle.
 
-    a_q [M,K/2], a_sf_lin [M,K/16], w_q [N,K/2], w_sf_lin [N,K/16]; g's are scalars.
+    a_q [M,K/2], a_sf_lin [M,K/16], w_q [N,K/2], w_sf_lin [N,K/16]; w_g is a scalar; a_g is a
+    scalar or, for an activation quantized per token, an array of M row scales.
     Returns fp16 bits [M,N] (uint16), plus the fp64 sums when want_f64.
     """
-    da = dequantize(a_q, a_sf_lin, a_g)
+    if np.ndim(a_g) > 0 and np.size(a_g) == np.shape(a_q)[0] and np.size(a_g) > 1:
+        da = dequantize_rows(a_q, a_sf_lin, a_g)
+    else:
+        da = dequantize(a_q, a_sf_lin, float(np.asarray(a_g).reshape(-1)[0]))
     dw = dequantize(w_q, w_sf_lin, w_g)
     out64 = np.matmul(da, dw.T)
     out16 = f64_to_f16(out64.reshape(-1)).reshape(out64.shape)

@@ -454,6 +454,18 @@ void orc_dequantize(const uint8_t *q, const uint8_t *s, float g, int64_t rows, i
           elem_value(q + r * (K / 2), k) * orc_e4m3_value(s[r * (K / 16) + k / 16]) / (double)g;
 }
 
+/*
+ * The same with one encode scale per row (an operand quantized per token): out[r, k] =
+ * E2M1(q[r, k]) * E4M3(s[r, k/16]) / g[r].
+ */
+void orc_dequantize_rows(const uint8_t *q, const uint8_t *s, const float *g, int64_t rows,
+                         int64_t K, double *out) {
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t k = 0; k < K; ++k)
+      out[r * K + k] = elem_value(q + r * (K / 2), k) * orc_e4m3_value(s[r * (K / 16) + k / 16]) /
+                       (double)g[r];
+}
+
 /* ------------------------------------------------------------------------------------ */
 /* Array helpers for the pin tests (elementwise loops over the scalar definitions).       */
 /* ------------------------------------------------------------------------------------ */

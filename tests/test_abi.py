@@ -88,8 +88,9 @@ def test_swiglu_argument_checks(L):
     assert f(P16, 0, 0, 32, 64, None, None, None, 1, None) == nv.OK
 
 
-def test_gemm_argument_checks(L):
-    g = L.nvfp4_gemm
+@pytest.mark.parametrize("entry", ["nvfp4_gemm", "nvfp4_gemm_per_token"])
+def test_gemm_argument_checks(L, entry):
+    g = getattr(L, entry)
     a = (P16, P16, 1, P16, P16, P16, P16, P16)
     assert g(*a, 16, 256, 96, None, 0, None, None) == nv.ERR_INVALID_ARG        # K % 64
     assert g(*a, 16, 250, 512, None, 0, None, None) == nv.ERR_INVALID_ARG       # N % 8

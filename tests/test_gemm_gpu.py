@@ -141,3 +141,53 @@ def test_gemm_prefill_workload():
     _, ref = orc.gemm(aq[rows], sa[rows], ga, wq[cols], ws[cols], gw, want_f64=True)
     gemm_close(got[np.ix_(rows, cols)], ref)
     assert np.isfinite(got.view(np.float16)).all()
+
+
+@pytest.mark.parametrize("M,N,K", [(8, 512, 1024), (32, 20480, 1024), (100, 520, 512),
+                                   (300, 264, 1024), (1024, 1024, 2048)])
+def test_gemm_per_token_activation_scales(M, N, K):
+    """Activation quantized per token (one g per row, as nvfp4_quantize(per_token=True)
+    writes), weights per tensor: nvfp4_gemm_per_token against the oracle GEMM with row
+    scales. Shapes reach the decode (M <= 32), single-CTA and CTA-pair kernels."""
+    nv = require_cuda()
+    a = workloads.per_token(M, K, seed=M + K)
+    w = workloads.normal((N, K), 0.02, seed=N + 3)
+    ab, wb = workloads.bits16(a), workloads.bits16(w)
+    a_q, a_sf, g_rows = orc.quantize(ab, per_token=True)
+    gw = orc.global_scale(wb)
+    w_q, w_sf, _ = orc.quantize(wb, g=gw)
+    _, ref = orc.gemm(a_q, a_sf, g_rows, w_q, w_sf, gw, want_f64=True)
+    layouts = [orc.L128x4, orc.L8x4] if M <= 32 else [orc.L128x4]
+    for layout in layouts:
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        out = nv.nvfp4_gemm(torch.from_numpy(a_q).cuda(),
+                            torch.from_numpy(orc.swizzle(a_sf, layout)).cuda(),
+                            torch.from_numpy(np.ascontiguousarray(g_rows)).cuda(),
+                            torch.from_numpy(w_q).cuda(),
+                            torch.from_numpy(orc.swizzle(w_sf, orc.L128x4)).cuda(),
+                            torch.tensor([gw], dtype=torch.float32, device="cuda"),
+                            a_layout=layout, dev_status=status, per_token_a=True)
+        torch.cuda.synchronize()
+        assert status.item() == 0
+        gemm_close(out.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+def test_per_token_quantize_then_gemm_pipeline():
+    """The whole per-token path on the GPU (quantize with per-row g, then the GEMM with those
+    row scales) against the same two steps in the oracle, from the same bf16 inputs."""
+    nv = require_cuda()
+    M, N, K = 384, 768, 2048
+    a = workloads.per_token(M, K, seed=77)
+    w = workloads.normal((N, K), 0.02, seed=78)
+    ab, wb = workloads.bits16(a), workloads.bits16(w)
+    a_q, a_sf, g_rows = orc.quantize(ab, per_token=True)
+    gw = orc.global_scale(wb)
+    w_q, w_sf, _ = orc.quantize(wb, g=gw)
+    _, ref = orc.gemm(a_q, a_sf, g_rows, w_q, w_sf, gw, want_f64=True)
+    ad, wd = a.cuda(), w.cuda()
+    aq_d, asf_d, ag_d = nv.nvfp4_quantize(ad, per_token=True, sf_layout=nv.SF_128x4)
+    gw_d = nv.nvfp4_global_scale(wd)
+    wq_d, wsf_d, _ = nv.nvfp4_quantize(wd, gw_d, sf_layout=nv.SF_128x4)
+    out = nv.nvfp4_gemm(aq_d, asf_d, ag_d, wq_d, wsf_d, gw_d, per_token_a=True)
+    torch.cuda.synchronize()
+    gemm_close(out.cpu().view(torch.int16).numpy().view(np.uint16), ref)

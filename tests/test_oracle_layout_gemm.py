@@ -192,3 +192,28 @@ def test_byte_counts_from_shapes(orc):
     assert f4 == 4 * NH + NH // 2 + NH // 16 == 267911168
     # the fused SwiGLU + NVFP4 workload moves 4.5625 NH bytes
     assert f4 / NH == 4.5625
+
+
+def test_gemm_per_row_activation_scales(orc):
+    """Per-token activation scales: with every row scale equal it is the scalar GEMM, and
+    otherwise output row m is the unit-scale GEMM's row divided by g[m] (the scale factors
+    out of the sum, so the fp64 results agree to rounding)."""
+    rng = np.random.default_rng(11)
+    M, N, K = 6, 40, 96
+    a = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    w = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = rng.integers(0x28, 0x48, (M, K // 16), dtype=np.uint8)
+    sw = rng.integers(0x28, 0x48, (N, K // 16), dtype=np.uint8)
+    g_rows = np.array([0.5, 3.0, 17.25, 1.0, 250.0, 0.125], np.float32)
+    same = np.full(M, 7.5, np.float32)
+    _, ref_same = orc.gemm(a, sa, 7.5, w, sw, 2.0, want_f64=True)
+    _, got_same = orc.gemm(a, sa, same, w, sw, 2.0, want_f64=True)
+    np.testing.assert_array_equal(got_same, ref_same)
+    _, unit = orc.gemm(a, sa, 1.0, w, sw, 2.0, want_f64=True)
+    _, rows = orc.gemm(a, sa, g_rows, w, sw, 2.0, want_f64=True)
+    np.testing.assert_allclose(rows, unit / g_rows[:, None].astype(np.float64), rtol=1e-12, atol=0)
+    # and against the triple loop, one row at a time with that row's scalar scale
+    for m in range(M):
+        _, loop_m = orc.gemm_loops(a[m:m + 1], sa[m:m + 1], float(g_rows[m]), w, sw, 2.0,
+                                   want_f64=True)
+        np.testing.assert_allclose(rows[m:m + 1], loop_m, rtol=1e-12, atol=1e-300)
