@@ -51,6 +51,10 @@ def algorithmic(workload, M=None, K=None, N=None, H=None, a_layout="128x4"):
         sf = (-(-M // 128) * 128) * (-(-(K // 16) // 4) * 4)
         g = M * 4
         return {"bytes": x + q + sf + g, "read": x, "written": q + sf + g, "flops": 0}
+    if workload == "swiglu_fp8":
+        x = M * 2 * H * 2
+        q = M * H
+        return {"bytes": x + q, "read": x, "written": q, "flops": 0}
     if workload == "swiglu":
         x = M * 2 * H * 2
         q = M * H // 2
@@ -222,6 +226,23 @@ def run_ours(args, rank, world, torch, dist):
                          "input": "bf16", "dist": "N(0,1)", "scales": "E4M3 128x4",
                          "global_scale": "fp32 per tensor", "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
         unit, factor = "GB/s", alg["bytes"] / 1e9
+    elif wl == "swiglu_fp8":
+        M, H = 4096, 14336
+        x_host = workloads.swiglu(M, H, seed=workloads.SEEDS["swiglu"] + rank)
+        copies = [x_host.to(dev) for _ in range(2)]
+        sdev = torch.tensor([448.0 / 60.0], dtype=torch.float32, device=dev)
+        q = torch.empty(M, H, dtype=torch.uint8, device=dev)
+        sf = torch.empty(1, dtype=torch.uint8, device=dev)
+        alg = algorithmic(wl, M=M, H=H)
+        kernel_key, kernel_name = "swiglu_fp8", "swiglu_fp8_kernel"
+
+        def step(i):
+            nv.swiglu_fp8_quantize(copies[i % 2], sdev, q=q)
+        launches_per_step, period = 1, 2
+        workload_desc = {"workload": "fused SwiGLU + FP8 E4M3 quantize", "shape": [M, 2 * H],
+                         "input": "bf16", "dist": "N(0,1)", "output": "E4M3 [M, H], scale 448/60",
+                         "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
+        unit, factor = "GB/s", alg["bytes"] / 1e9
     elif wl in ("decode", "prefill", "tiny"):
         if wl == "decode":
             M, N, K = args.m, 28672, 8192
@@ -323,12 +344,12 @@ def run_ours(args, rank, world, torch, dist):
 
     # ---- end to end through the public API with host buffers (pinned), copies timed
     e2e = None
-    if wl in ("per_token", "swiglu"):
+    if wl in ("per_token", "swiglu", "swiglu_fp8"):
         src = copies[0]
         h_in = torch.empty(src.shape, dtype=src.dtype, pin_memory=True)
         h_in.copy_(src.cpu())
         h_q = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-        h_sf = torch.empty(sf.shape, dtype=sf.dtype, pin_memory=True)
+        h_sf = torch.empty(sf.shape, dtype=sf.dtype, pin_memory=True) if wl != "swiglu_fp8" else None
         h_g = torch.empty(g.shape, dtype=g.dtype, pin_memory=True) if wl == "per_token" else None
         d_in = torch.empty_like(src)
 
@@ -337,10 +358,13 @@ def run_ours(args, rank, world, torch, dist):
             if wl == "per_token":
                 nv.nvfp4_quantize(d_in, g, per_token=True, sf_layout=nv.SF_128x4, q=q, sf=sf)
                 h_g.copy_(g, non_blocking=True)
-            else:
+            elif wl == "swiglu":
                 nv.swiglu_nvfp4_quantize(d_in, gdev, sf_layout=nv.SF_128x4, q=q, sf=sf)
+            else:
+                nv.swiglu_fp8_quantize(d_in, sdev, q=q)
             h_q.copy_(q, non_blocking=True)
-            h_sf.copy_(sf, non_blocking=True)
+            if h_sf is not None:
+                h_sf.copy_(sf, non_blocking=True)
 
         for _ in range(2):
             e2e_step()
@@ -357,7 +381,7 @@ def run_ours(args, rank, world, torch, dist):
             tt = torch.tensor([e2e_ms], device=dev)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             e2e_ms = tt.item()
-        d2h = h_q.numel() + h_sf.numel() + (h_g.numel() * 4 if h_g is not None else 0)
+        d2h = h_q.numel() + (h_sf.numel() if h_sf is not None else 0) + (h_g.numel() * 4 if h_g is not None else 0)
         e2e = {"value": world * factor / (e2e_ms / 1e3), "unit": unit,
                "h2d_bytes_per_step": h_in.numel() * 2, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms}
@@ -450,6 +474,13 @@ def _oracle_sample(wl, args):
         alg = algorithmic("swiglu", M=rows, H=14336)
         return (lambda: oracle.swiglu_quantize(bits, g, oracle.BF16)), alg["bytes"] / 1e9, \
             f"{rows} of 4096 rows", "GB/s"
+    if wl == "swiglu_fp8":
+        rows = max(1, args.cpu_rows // 2)
+        x = workloads.swiglu(rows, 14336)
+        bits = workloads.bits16(x)
+        alg = algorithmic("swiglu_fp8", M=rows, H=14336)
+        return (lambda: oracle.swiglu_fp8(bits, 448.0 / 60.0, oracle.BF16)), alg["bytes"] / 1e9, \
+            f"{rows} of 4096 rows", "GB/s"
     if wl in ("decode", "prefill", "tiny"):
         if wl == "decode":
             M, N, K = args.m, 512, 8192
@@ -492,7 +523,7 @@ def cpu_baseline(wl, args):
     t = time.perf_counter()
     fn()
     dt = time.perf_counter() - t
-    cores = 1 if wl in ("per_token", "swiglu") else _threads_used()
+    cores = 1 if wl in ("per_token", "swiglu", "swiglu_fp8") else _threads_used()
     return {"value": units / dt, "unit": unit, "cores": cores, "kind": "oracle",
             "sample": desc, "seconds": dt}
 
@@ -507,7 +538,7 @@ def run_reference(args, rank, world):
     for _ in range(args.steps):
         fn()
     dt = (time.perf_counter() - t) / args.steps
-    cores = 1 if args.workload in ("per_token", "swiglu") else _threads_used()
+    cores = 1 if args.workload in ("per_token", "swiglu", "swiglu_fp8") else _threads_used()
     value = units / dt
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
@@ -528,7 +559,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="per_token",
-                    choices=["per_token", "swiglu", "decode", "prefill", "tiny"])
+                    choices=["per_token", "swiglu", "swiglu_fp8", "decode", "prefill", "tiny"])
     ap.add_argument("--m", type=int, default=32, help="tokens of the decode workload")
     ap.add_argument("--a-layout", default="128x4", choices=["128x4", "8x4"])
     ap.add_argument("--cpu-rows", type=int, default=2048)

@@ -165,6 +165,21 @@ NVFP4_API int swiglu_nvfp4_quantize(const void *x, int dtype, int64_t M, int64_t
                           const float *g, uint8_t *q, uint8_t *sf, int sf_layout, void *stream);
 
 /*
+ * Fused SwiGLU + FP8 E4M3 quantize, the kernel of "Building Custom TensorRT-LLM Plugins for
+ * Low-Latency FP8 Inference at Scale" ("Fusing the Kernel in CUDA"; plugin I/O: BF16/FP16
+ * [N, 2H] activations, an fp32 scale, FP8 E4M3 [N, H] output in linear layout):
+ *   q[r, h] = E4M3( fp32(silu(gate) * up) * scale ), round to nearest even, saturating to
+ *   +-448, NaN -> 0x7F; silu and its exponential exactly as in swiglu_nvfp4_quantize.
+ * x      device, [M, 2H] bf16/fp16 row-major (gate = columns [0, H), up = [H, 2H)), row
+ *        stride ldx >= 2H elements, 16-byte aligned rows.
+ * scale  device fp32 [1]: multiplies y (a static calibration scale, or 448 / amax(y)).
+ * q      device, [M, H] bytes, row-major, 16-byte aligned.
+ * Requires H % 16 == 0. Y is never written to memory: 4NH bytes read + NH written.
+ */
+NVFP4_API int swiglu_fp8_quantize(const void *x, int dtype, int64_t M, int64_t H, int64_t ldx,
+                                  const float *scale, uint8_t *q, void *stream);
+
+/*
  * Scale-layout conversion (the 128x4 / 8x4 layouts of "feature: add fp4 mm using trtllm
  * backend", FlashInfer PR #1355, description item 1; weight/scale preparation).
  * nvfp4_sf_swizzle:   lin [R, C] bytes (row-major)  ->  out in `layout` (padding zeroed).

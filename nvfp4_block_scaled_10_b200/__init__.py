@@ -33,6 +33,7 @@ SIGNATURES = {
     "nvfp4_global_scale_noalloc": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_quantize": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _i32, _vp]),
     "swiglu_nvfp4_quantize": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp, _i32, _vp]),
+    "swiglu_fp8_quantize": (_i32, [_vp, _i32, _i64, _i64, _i64, _vp, _vp, _vp]),
     "nvfp4_sf_swizzle": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
     "nvfp4_sf_unswizzle": (_i32, [_vp, _vp, _i64, _i64, _i32, _vp]),
     "nvfp4_gemm_workspace_bytes": (_sz, [_i64, _i64, _i64]),
@@ -176,6 +177,19 @@ def swiglu_nvfp4_quantize(x: torch.Tensor, g: torch.Tensor, sf_layout: int = SF_
                                        _ptr(sf), sf_layout, _stream(stream)),
            "swiglu_nvfp4_quantize")
     return q, sf
+
+
+def swiglu_fp8_quantize(x: torch.Tensor, scale: torch.Tensor, q: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """Fused silu(gate) * up -> FP8 E4M3 (saturating) for x [M, 2H] = [gate | up]; returns
+    q uint8 [M, H] (E4M3 bit patterns). scale: device fp32 [1], multiplies y."""
+    M, H2, ldx = _rows_ld(x)
+    H = H2 // 2
+    if q is None:
+        q = torch.empty(M, H, dtype=torch.uint8, device=x.device)
+    _check(lib().swiglu_fp8_quantize(_ptr(x), _dtype_code(x), M, H, ldx, _ptr(scale), _ptr(q),
+                                     _stream(stream)), "swiglu_fp8_quantize")
+    return q
 
 
 def nvfp4_sf_swizzle(lin: torch.Tensor, layout: int = SF_128x4, out: torch.Tensor | None = None,

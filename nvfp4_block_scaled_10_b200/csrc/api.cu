@@ -151,6 +151,19 @@ int swiglu_nvfp4_quantize(const void *x, int dtype, int64_t M, int64_t H, int64_
                                        d->num_sms, static_cast<cudaStream_t>(stream)));
 }
 
+int swiglu_fp8_quantize(const void *x, int dtype, int64_t M, int64_t H, int64_t ldx,
+                        const float *scale, uint8_t *q, void *stream) {
+  int s = check_activation(x, dtype, M, H, ldx, 2 * H);
+  if (s != NVFP4_OK) return s;
+  if (M == 0) return NVFP4_OK;
+  if (scale == nullptr || q == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(q) || (reinterpret_cast<uintptr_t>(scale) & 3u) != 0) return NVFP4_ERR_MISALIGNED;
+  const DeviceInfo *d = device_info();
+  if (d == nullptr) return NVFP4_ERR_CUDA;
+  return finish(launch_swiglu_fp8(x, dtype, M, H, ldx, scale, q, d->num_sms,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
 int nvfp4_sf_swizzle(const uint8_t *lin, uint8_t *out, int64_t R, int64_t C, int layout,
                      void *stream) {
   if (!valid_layout(layout) || R < 0 || C < 0) return NVFP4_ERR_INVALID_ARG;

@@ -27,6 +27,8 @@ cudaError_t launch_quantize(const void *x, int dtype, int64_t M, int64_t K, int6
 cudaError_t launch_swiglu_quantize(const void *x, int dtype, int64_t M, int64_t H, int64_t ldx,
                                    const float *g, uint8_t *q, uint8_t *sf, int layout, int64_t Rp,
                                    int64_t Cp, int num_sms, cudaStream_t st);
+cudaError_t launch_swiglu_fp8(const void *x, int dtype, int64_t M, int64_t H, int64_t ldx,
+                              const float *scale, uint8_t *q, int num_sms, cudaStream_t st);
 cudaError_t launch_sf_swizzle(const uint8_t *lin, uint8_t *out, int64_t R, int64_t C, int layout,
                               int64_t Rp, int64_t Cp, int num_sms, cudaStream_t st);
 cudaError_t launch_sf_unswizzle(const uint8_t *in, uint8_t *lin, int64_t R, int64_t C, int layout,

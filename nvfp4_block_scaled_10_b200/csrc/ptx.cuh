@@ -359,6 +359,14 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float v) {
   return static_cast<uint32_t>(out) & 0xFFu;
 }
 
+// Two fp32 -> two signed E4M3 codes, lo in the low byte (round to nearest even, saturate to
+// +-448, NaN -> NaN).
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+  return static_cast<uint32_t>(out);
+}
+
 // E4M3 code -> fp32 (exact: every E4M3 value is an fp16 value).
 __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   uint32_t h2;

@@ -496,6 +496,67 @@ __global__ void __launch_bounds__(NT, MINB) swiglu_quant_kernel(
   zero_sf_padding(sf, layout, M, C, Rp, Cp);
 }
 
+// Fused SwiGLU + FP8 E4M3, the write-up's own kernel ("Building Custom TensorRT-LLM Plugins for
+// Low-Latency FP8 Inference at Scale", "Fusing the Kernel in CUDA"): q = E4M3(fl(y * scale)),
+// saturating at +-448, y = silu(gate) * up in fp32 exactly as in the NVFP4 variant; q is
+// [M, H] row-major, one 16-byte store per 16-element block. Same work items and rolling
+// next-item loads as swiglu_quant_kernel.
+template <int DTYPE, int UNROLL, bool V8, int NT, int MINB>
+__global__ void __launch_bounds__(NT, MINB) swiglu_fp8_kernel(
+    const uint16_t *__restrict__ x, int64_t M, int64_t H, int64_t ldx,
+    const float *__restrict__ scale, uint8_t *__restrict__ q, int chunks_per_row) {
+  const int C = static_cast<int>(H / 16);
+  const float sc = scale[0];
+  const int64_t step_r = gridDim.x / chunks_per_row;
+  const int step_ch = static_cast<int>(gridDim.x % chunks_per_row);
+  int64_t r = blockIdx.x / chunks_per_row;
+  int ch = static_cast<int>(blockIdx.x % chunks_per_row);
+  uint32_t wg[UNROLL][8], wu[UNROLL][8];
+  if (r < M) load_swiglu_item<DTYPE, UNROLL, V8>(x, ldx, H, C, r, ch * (NT * UNROLL) + threadIdx.x, NT, wg, wu);
+  while (r < M) {
+    int64_t rn = r + step_r;
+    int chn = ch + step_ch;
+    if (chn >= chunks_per_row) {
+      chn -= chunks_per_row;
+      ++rn;
+    }
+    const int c0 = ch * (NT * UNROLL) + static_cast<int>(threadIdx.x);
+    const int c0n = chn * (NT * UNROLL) + static_cast<int>(threadIdx.x);
+    const uint16_t *gnext = x + rn * ldx;
+    uint8_t *qrow = q + r * H;
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int c = c0 + u * NT;
+      float y[16];
+      if (c < C) {
+        const float gmax = amax16_packed<DTYPE>(wg[u]);
+        if (gmax <= 87.0f) swiglu_block16<DTYPE, false, false>(wg[u], wu[u], y);
+        else if (gmax != INFINITY) swiglu_block16<DTYPE, true, false>(wg[u], wu[u], y);
+        else swiglu_block16<DTYPE, true, true>(wg[u], wu[u], y);
+      }
+      const int cn = c0n + u * NT;
+      if (rn < M && cn < C) {
+        ld_block16<V8>(gnext + cn * 16, wg[u]);
+        ld_block16<V8>(gnext + H + cn * 16, wu[u]);
+      }
+      if (c < C) {
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const F2 a = mul2f_rn(F2{y[4 * k], y[4 * k + 1]}, F2{sc, sc});
+          const F2 b = mul2f_rn(F2{y[4 * k + 2], y[4 * k + 3]}, F2{sc, sc});
+          o[k] = cvt_e4m3x2(a.x, a.y) | (cvt_e4m3x2(b.x, b.y) << 16);
+        }
+        asm volatile("st.global.cs.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(qrow + c * 16), "r"(o[0]),
+                     "r"(o[1]), "r"(o[2]), "r"(o[3])
+                     : "memory");
+      }
+    }
+    r = rn;
+    ch = chn;
+  }
+}
+
 // ------------------------------------------------------------------------------ layouts
 
 __global__ void sf_swizzle_kernel(const uint8_t *__restrict__ lin, uint8_t *__restrict__ out,
@@ -657,6 +718,22 @@ cudaError_t launch_swiglu_quantize(const void *x, int dtype, int64_t M, int64_t 
                        (swiglu_quant_kernel<DT, kUnroll, VV, kNT, kMinB>
                         <<<static_cast<int>(grid), kNT, 0, st>>>(xp, M, H, ldx, g, q, sf, layout,
                                                                  Rp, Cp, cpr)));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_swiglu_fp8(const void *x, int dtype, int64_t M, int64_t H, int64_t ldx,
+                              const float *scale, uint8_t *q, int num_sms, cudaStream_t st) {
+  const uint16_t *xp = static_cast<const uint16_t *>(x);
+  constexpr int kNT = 224, kUnroll = 2, kMinB = 4;
+  const int64_t C = H / 16;
+  const int cpr = static_cast<int>((C + kNT * kUnroll - 1) / (kNT * kUnroll));
+  int64_t grid = static_cast<int64_t>(num_sms) * kMinB;
+  if (grid > M * cpr) grid = M * cpr;
+  if (grid < 1) grid = 1;
+  const bool v8 = blocks_32b_aligned(x, ldx);
+  NVFP4_DISPATCH_DT_V8(dtype, v8,
+                       (swiglu_fp8_kernel<DT, kUnroll, VV, kNT, kMinB>
+                        <<<static_cast<int>(grid), kNT, 0, st>>>(xp, M, H, ldx, scale, q, cpr)));
   return cudaGetLastError();
 }
 

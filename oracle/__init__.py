@@ -79,6 +79,8 @@ def lib():
             "orc_gemm": (None, [vp, vp, f32, vp, vp, f32, i64, i64, i64, vp, vp]),
             "orc_dequantize": (None, [vp, vp, f32, i64, i64, vp]),
             "orc_dequantize_rows": (None, [vp, vp, vp, i64, i64, vp]),
+            "orc_swiglu_fp8": (None, [vp, i32, i64, i64, i64, f32, vp]),
+            "orc_e4m3_encode_signed_array": (None, [vp, i64, vp]),
             "orc_e2m1_encode_array": (None, [vp, i64, vp]),
             "orc_e4m3_encode_array": (None, [vp, i64, vp]),
             "orc_exp_array": (None, [vp, i64, vp]),
@@ -220,6 +222,24 @@ def swiglu_amax(x_bits: np.ndarray, dtype: int = BF16) -> float:
     x = _c(x_bits, np.uint16)
     M, H2 = x.shape
     return float(np.float32(lib().orc_swiglu_amax(_p(x), dtype, M, H2 // 2, H2)))
+
+
+def e4m3_encode_signed(v) -> np.ndarray:
+    """Signed saturating FP8 E4M3 codes of fp32 values (NaN -> 0x7F)."""
+    vv = _c(np.atleast_1d(v), np.float32)
+    out = np.empty(vv.shape, np.uint8)
+    lib().orc_e4m3_encode_signed_array(_p(vv), vv.size, _p(out))
+    return out
+
+
+def swiglu_fp8(x_bits: np.ndarray, scale: float, dtype: int = BF16) -> np.ndarray:
+    """Fused SwiGLU + FP8 E4M3: q [M, H] = E4M3_sat(fl(silu(gate) * up) * scale)."""
+    x = _c(x_bits, np.uint16)
+    M, H2 = x.shape
+    H = H2 // 2
+    q = np.zeros((M, H), np.uint8)
+    lib().orc_swiglu_fp8(_p(x), dtype, M, H, H2, float(np.float32(scale)), _p(q))
+    return q
 
 
 def swiglu_quantize(x_bits: np.ndarray, g: float, dtype: int = BF16):

@@ -340,6 +340,37 @@ void orc_swiglu_quantize(const uint16_t *x, int dtype, int64_t M, int64_t H, int
     }
 }
 
+/*
+ * FP8 E4M3 with sign (OCP OFP8 E4M3): NaN -> 0x7F; otherwise the sign bit (bit 7, kept for
+ * -0 and for negatives that round to zero) and the saturating magnitude code of |v|, round
+ * to nearest even, |v| >= 448 (infinity included) -> 448.
+ */
+int orc_e4m3_encode_signed(float v) {
+  if (v != v) return 0x7F;
+  const int sign = signbit(v) ? 0x80 : 0;
+  return sign | orc_e4m3_encode(fabsf(v));
+}
+
+/*
+ * Fused SwiGLU + FP8 E4M3 quantize ("Building Custom TensorRT-LLM Plugins for Low-Latency FP8
+ * Inference at Scale", "Fusing the Kernel in CUDA": SwiGLU in fp32, the quantization scale
+ * applied, saturation to +-448): q[r, h] = E4M3(fl(y[r, h] * scale)), y = silu(gate) * up in
+ * fp32, q [M, H] row-major. The scale multiplies, as the NVFP4 encode scales do here.
+ */
+void orc_swiglu_fp8(const uint16_t *x, int dtype, int64_t M, int64_t H, int64_t ldx, float scale,
+                    uint8_t *q) {
+  for (int64_t r = 0; r < M; ++r)
+    for (int64_t h = 0; h < H; ++h) {
+      const float y =
+          orc_swiglu_elem(load_elem(x, dtype, r * ldx + h), load_elem(x, dtype, r * ldx + H + h));
+      q[r * H + h] = (uint8_t)orc_e4m3_encode_signed(y * scale);
+    }
+}
+
+void orc_e4m3_encode_signed_array(const float *v, int64_t n, uint8_t *out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = (uint8_t)orc_e4m3_encode_signed(v[i]);
+}
+
 /* amax of Y = silu(gate) * up (used to pick the per-tensor g for the fused kernel). */
 float orc_swiglu_amax(const uint16_t *x, int dtype, int64_t M, int64_t H, int64_t ldx) {
   float amax = 0.0f;

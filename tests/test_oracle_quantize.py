@@ -164,3 +164,61 @@ def test_swiglu_zero_gate(orc):
     assert (orc.swiglu(workloads.bits16(x)) == 0).all()
     q, s = orc.swiglu_quantize(workloads.bits16(x), 1.0)
     assert (q == 0).all() and (s == 0).all()
+
+
+# ------------------------------------------------------------------------------ SwiGLU + FP8
+
+
+def _e4m3_decode(codes):
+    """Value of signed E4M3 codes (OCP OFP8: bias 7, subnormals at exponent 0, 0x7F NaN)."""
+    c = np.asarray(codes, np.int64)
+    e, m = (c >> 3) & 15, c & 7
+    mag = np.where(e > 0, (1.0 + m / 8.0) * 2.0 ** (e - 7.0), (m / 8.0) * 2.0 ** -6)
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return np.where(c & 0x80, -mag, mag)
+
+
+def test_e4m3_signed_encoder(orc):
+    v = np.float32(np.concatenate([np.linspace(0, 470, 20001), [1e-9, 0.0019, 2 ** -9, 1e30, np.inf]]))
+    pos = orc.e4m3_encode_signed(v)
+    assert np.array_equal(pos, orc.e4m3_encode(v))                   # magnitudes: the scale encoder
+    neg = orc.e4m3_encode_signed(-v)
+    assert np.array_equal(neg, pos | 0x80)                            # sign bit, -0 included
+    assert orc.e4m3_encode_signed(np.float32(np.nan))[0] == 0x7F
+    # against torch's float8_e4m3fn cast (round to nearest even) where no saturation applies
+    import torch
+    w = np.float32(np.random.default_rng(3).uniform(-463, 463, 50000))
+    t = torch.from_numpy(w).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(orc.e4m3_encode_signed(w), t)
+
+
+def test_swiglu_fp8_bounds_and_saturation(orc):
+    """q = E4M3_sat(y * scale): decode(q) is within half an E4M3 step of y * scale below 448,
+    exactly +-448 at or above, and the sign of y is kept (zero included)."""
+    from nvfp4_block_scaled_10_b200 import workloads
+    x = workloads.swiglu(8, 64, seed=9)
+    bits = workloads.bits16(x)
+    for scale in (1.0, 37.0, 900.0):
+        q = orc.swiglu_fp8(bits, scale)
+        y = orc.swiglu(bits).astype(np.float64)
+        t = np.float32(y * scale).astype(np.float64)  # one fp32 product, as defined
+        d = _e4m3_decode(q)
+        big = np.abs(t) >= 448
+        assert np.all(np.abs(d[big]) == 448.0) and np.all(np.sign(d[big]) == np.sign(t[big]))
+        small = ~big
+        # half a step: the E4M3 spacing at |t| is 2^(floor(log2|t|) - 3), subnormals 2^-9
+        ex = np.floor(np.log2(np.maximum(np.abs(t[small]), 2.0 ** -6)))
+        half = 2.0 ** (ex - 3) / 2
+        assert np.all(np.abs(d[small] - t[small]) <= half + 1e-30)
+        assert np.all((q[small] & 0x80 != 0) == np.signbit(t[small]))
+
+
+def test_swiglu_fp8_traffic_reading(orc):
+    """The fused SwiGLU + FP8 call reads X and writes Q only: its input and output buffers add
+    up to the fused byte count recomputed from the shapes (5NH), not to the printed 9NH."""
+    from nvfp4_block_scaled_10_b200 import workloads
+    N, H = 16, 64
+    bits = workloads.bits16(workloads.swiglu(N, H, seed=4))
+    q = orc.swiglu_fp8(bits, 1.0)
+    _, fused = orc.swiglu_quant_traffic_from_shapes(N, H, out="fp8")
+    assert bits.nbytes + q.nbytes == fused == 5 * N * H

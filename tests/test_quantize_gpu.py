@@ -250,3 +250,48 @@ def test_tiny_workload_quantize():
             torch.cuda.synchronize()
             assert_bytes_equal(host_bytes(q), q_o, "q")
             assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, layout), "sf")
+
+
+# ------------------------------------------------------------------------------ SwiGLU + FP8
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("M,H,pad,scale", [(1, 16, 0, 1.0), (5, 48, 8, 37.0), (130, 1040, 16, 3.0),
+                                           (64, 14336, 0, 448.0 / 60.0), (3, 512, 0, 5000.0)])
+def test_swiglu_fp8_parity(M, H, pad, scale, dtype):
+    nv = require_cuda()
+    tdt, odt = DT[dtype]
+    x = workloads.normal((M, 2 * H + pad), 1.0, seed=M + H, dtype=tdt)
+    xs = x[:, :2 * H].contiguous()
+    q_o = orc.swiglu_fp8(workloads.bits16(xs), scale, odt)
+    q = nv.swiglu_fp8_quantize(x.cuda()[:, :2 * H], torch.tensor([scale], device="cuda"))
+    torch.cuda.synchronize()
+    assert_bytes_equal(host_bytes(q), q_o, "q")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_swiglu_fp8_special_values(dtype):
+    # infinite gates and ups (saturation to +-448), NaN (0x7F), signed zeros, tiny values
+    nv = require_cuda()
+    tdt, odt = DT[dtype]
+    inf, nan = float("inf"), float("nan")
+    gate = torch.tensor([[inf, -inf, -0.0, 0.0, 1.5, -2.0, 3e-5, -3e-5, 7.0, -7.0, 60.0, 1.0,
+                          nan, 2.0, -3.0, 4.0]], dtype=torch.float32)
+    up = torch.tensor([[2.0, 2.0, 1.0, -1.0, inf, -inf, 1.0, 1.0, 1e4, 1e4, -100.0, nan,
+                        1.0, 0.0, -0.0, 0.5]], dtype=torch.float32)
+    x = torch.cat([gate, up], dim=1).to(tdt)
+    for scale in [1.0, 10.0]:
+        q_o = orc.swiglu_fp8(workloads.bits16(x), scale, odt)
+        q = nv.swiglu_fp8_quantize(x.cuda(), torch.tensor([scale], device="cuda"))
+        torch.cuda.synchronize()
+        assert_bytes_equal(host_bytes(q), q_o, "q")
+
+
+def test_swiglu_fp8_workload_full():
+    nv = require_cuda()
+    x = workloads.swiglu(4096, 14336)
+    scale = 448.0 / 60.0
+    q_o = orc.swiglu_fp8(workloads.bits16(x), scale, orc.BF16)
+    q = nv.swiglu_fp8_quantize(x.cuda(), torch.tensor([scale], device="cuda"))
+    torch.cuda.synchronize()
+    assert_bytes_equal(host_bytes(q), q_o, "q")
