@@ -60,9 +60,11 @@ def algorithmic(workload, M=None, K=None, N=None, H=None, a_layout="128x4"):
         q = M * H // 2
         sf = (-(-M // 128) * 128) * (-(-(H // 16) // 4) * 4)
         return {"bytes": x + q + sf, "read": x, "written": q + sf, "flops": 0}
-    if workload in ("decode", "prefill", "tiny"):
+    if workload in ("decode", "prefill", "tiny", "decode_f32"):
         rows_a = (-(-M // 8) * 8) if a_layout == "8x4" else (-(-M // 128) * 128)
         a = M * K // 2 + rows_a * K // 16
+        if workload == "decode_f32":  # fp32 activation scales [M, K/16]
+            a = M * K // 2 + M * (K // 16) * 4
         w = N * K // 2 + (-(-N // 128) * 128) * K // 16
         out = M * N * 2
         return {"bytes": a + w + out, "read": a + w, "written": out, "flops": 2 * M * N * K}
@@ -243,8 +245,8 @@ def run_ours(args, rank, world, torch, dist):
                          "input": "bf16", "dist": "N(0,1)", "output": "E4M3 [M, H], scale 448/60",
                          "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
         unit, factor = "GB/s", alg["bytes"] / 1e9
-    elif wl in ("decode", "prefill", "tiny"):
-        if wl == "decode":
+    elif wl in ("decode", "prefill", "tiny", "decode_f32"):
+        if wl in ("decode", "decode_f32"):
             M, N, K = args.m, 28672, 8192
             a_b, w_b = workloads.decode(M, N, K)
             ncopy = 2
@@ -262,25 +264,42 @@ def run_ours(args, rank, world, torch, dist):
         gw = nv.nvfp4_global_scale(w_d)
         ops = []
         for _ in range(ncopy):
-            aq, asf, _ = nv.nvfp4_quantize(a_d, ga, sf_layout=layout_code)
+            if wl == "decode_f32":
+                # the plugin contract: combined fp32 activation scales E4M3 x fp32(1 / ga) and a
+                # multiplying weight scale fp32(1 / gw) (input preparation, not timed)
+                aq, asf_lin, _ = nv.nvfp4_quantize(a_d, ga, sf_layout=nv.SF_LINEAR)
+                asf = (asf_lin.view(torch.float8_e4m3fn).float().view(M, K // 16)
+                       * (1.0 / ga)).contiguous()
+            else:
+                aq, asf, _ = nv.nvfp4_quantize(a_d, ga, sf_layout=layout_code)
             wq, wsf, _ = nv.nvfp4_quantize(w_d, gw, sf_layout=nv.SF_128x4)
             ops.append((aq, asf, wq, wsf))
         del a_d, w_d
+        w_scale = (1.0 / gw).contiguous()
         out = torch.empty(M, N, dtype=torch.float16, device=dev)
         alg = algorithmic(wl, M=M, N=N, K=K, a_layout=args.a_layout)
         kernel_key, kernel_name = f"gemm_{wl}", "gemm_nvfp4_kernel"
 
-        ws_bytes = nv.nvfp4_gemm_workspace_bytes(M, N, K)
+        if wl == "decode_f32":
+            ws_bytes = nv.nvfp4_gemm_act_f32_workspace_bytes(M, N, K)
+        else:
+            ws_bytes = nv.nvfp4_gemm_workspace_bytes(M, N, K)
         gemm_ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
 
+        def gemm_call(aq, asf, wq, wsf, ws):
+            if wl == "decode_f32":
+                nv.nvfp4_gemm_act_f32(aq, asf, wq, wsf, w_scale, out=out, workspace=ws)
+            else:
+                nv.nvfp4_gemm(aq, asf, ga, wq, wsf, gw, a_layout=layout_code, out=out, workspace=ws)
+
         def step(i):
-            aq, asf, wq, wsf = ops[i % ncopy]
-            nv.nvfp4_gemm(aq, asf, ga, wq, wsf, gw, a_layout=layout_code, out=out, workspace=gemm_ws)
+            gemm_call(*ops[i % ncopy], gemm_ws)
         launches_per_step, period = 1, ncopy
         workload_desc = {"workload": f"NVFP4 GEMM ({wl})", "M": M, "N": N, "K": K,
-                         "a_scales": args.a_layout, "w_scales": "128x4", "out": "fp16",
+                         "a_scales": "fp32 [M, K/16]" if wl == "decode_f32" else args.a_layout,
+                         "w_scales": "128x4", "out": "fp16",
                          "l2": f"operands rotated over {ncopy} copies"}
-        if wl == "decode":
+        if wl in ("decode", "decode_f32"):
             unit, factor = "GB/s", alg["bytes"] / 1e9
         else:
             unit, factor = "TFLOP/s", alg["flops"] / 1e12
@@ -385,7 +404,7 @@ def run_ours(args, rank, world, torch, dist):
         e2e = {"value": world * factor / (e2e_ms / 1e3), "unit": unit,
                "h2d_bytes_per_step": h_in.numel() * 2, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms}
-    elif wl in ("decode", "prefill", "tiny"):
+    elif wl in ("decode", "prefill", "tiny", "decode_f32"):
         aq, asf, wq, wsf = ops[0]
         hs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (aq, asf, wq, wsf)]
         for h, t in zip(hs, (aq, asf, wq, wsf)):
@@ -396,7 +415,7 @@ def run_ours(args, rank, world, torch, dist):
         def e2e_step():
             for d, h in zip(ds, hs):
                 d.copy_(h, non_blocking=True)
-            nv.nvfp4_gemm(ds[0], ds[1], ga, ds[2], ds[3], gw, a_layout=layout_code, out=out)
+            gemm_call(ds[0], ds[1], ds[2], ds[3], gemm_ws)
             h_out.copy_(out, non_blocking=True)
 
         for _ in range(2):
@@ -481,6 +500,19 @@ def _oracle_sample(wl, args):
         alg = algorithmic("swiglu_fp8", M=rows, H=14336)
         return (lambda: oracle.swiglu_fp8(bits, 448.0 / 60.0, oracle.BF16)), alg["bytes"] / 1e9, \
             f"{rows} of 4096 rows", "GB/s"
+    if wl == "decode_f32":
+        M, N, K = args.m, 512, 8192
+        a, w = workloads.decode(args.m, 28672, 8192)
+        ab, wb = workloads.bits16(a), workloads.bits16(w[:N])
+        ga, gw = oracle.global_scale(ab), oracle.global_scale(workloads.bits16(w))
+        aq, sa, _ = oracle.quantize(ab, g=ga)
+        wq, sw, _ = oracle.quantize(wb, g=gw)
+        table = np.array([oracle.e4m3_value(c) for c in range(256)], np.float64)
+        sa32 = np.float32(table[sa] * np.float64(np.float32(1.0 / ga)))
+        w_scale = float(np.float32(1.0 / gw))
+        alg = algorithmic("decode_f32", M=M, N=N, K=K)
+        return (lambda: oracle.gemm_act_f32(aq, sa32, wq, sw, w_scale)), alg["bytes"] / 1e9, \
+            f"M={args.m}, 512 of 28672 weight rows", "GB/s"
     if wl in ("decode", "prefill", "tiny"):
         if wl == "decode":
             M, N, K = args.m, 512, 8192
@@ -559,7 +591,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="per_token",
-                    choices=["per_token", "swiglu", "swiglu_fp8", "decode", "prefill", "tiny"])
+                    choices=["per_token", "swiglu", "swiglu_fp8", "decode", "decode_f32", "prefill",
+                             "tiny"])
     ap.add_argument("--m", type=int, default=32, help="tokens of the decode workload")
     ap.add_argument("--a-layout", default="128x4", choices=["128x4", "8x4"])
     ap.add_argument("--cpu-rows", type=int, default=2048)

@@ -248,6 +248,37 @@ NVFP4_API int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int 
                                    void *workspace, size_t workspace_bytes, int32_t *dev_status,
                                    void *stream);
 
+/*
+ * The GEMM under the activation contract of "Fused Nvfp4 GEMM All Reduce Plugin"
+ * (TensorRT-Edge-LLM C++ API, inputs [1] and [4]): the activation scales are combined FP32
+ * values [B,1,K/16] (the E4M3 block scale already multiplied by the activation's FP32
+ * dequantization scale) and the scalar FP32 weight scale multiplies (DequantizeLinear form):
+ *   out[m,n] = fp16( sum_k E2M1(a[m,k]) * sa32[m,k/16] * E2M1(w[n,k]) * E4M3(sw[n,k/16])
+ *                    * w_scale ).
+ * The block-scaled MMA takes E4M3 scales only, so the kernel splits each activation row's
+ * scales into three planes of E4M3 codes and one fp32 factor (rho = row maximum / 448):
+ * rho * (v1 + v2 + v3) is within 2^-12 of each scale relative. One MMA per K step takes the
+ * token rows once per plane (N = 96) and the epilogue adds the three fp32 partial sums. The
+ * split runs inside the GEMM kernel (one launch per 32 activation rows, in stream order).
+ * a_q      device, [M, K/2] packed E2M1, 16-byte aligned.
+ * a_sf32   device, fp32 [M, K/16] row-major (the [B,1,K/16] tensor), 16-byte aligned; every
+ *          scale finite and >= 0. A negative, NaN or infinite scale is an argument error the
+ *          kernel detects: its block counts as zero and 2 is ORed into *dev_status.
+ * w_q      device, [N, K/2] packed E2M1.   w_sf device, 128x4 layout (E4M3).
+ * w_scale  device, one fp32 (multiplies; 1 / the weight's encode scale).
+ * out      device, [M, N] fp16, row-major.
+ * workspace/workspace_bytes: device, 16-byte aligned, >= nvfp4_gemm_act_f32_workspace_bytes
+ *          (M, N, K); same use as in nvfp4_gemm.
+ * dev_status: device int32 or NULL; bit 1 a bounded wait gave up (NVFP4_ERR_TIMEOUT), bit 2
+ *          a bad activation scale. The caller reads it after synchronizing.
+ * Requires: K % 64 == 0, N % 8 == 0.
+ */
+NVFP4_API size_t nvfp4_gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K);
+NVFP4_API int nvfp4_gemm_act_f32(const uint8_t *a_q, const float *a_sf32, const uint8_t *w_q,
+                                 const uint8_t *w_sf, const float *w_scale, void *out, int64_t M,
+                                 int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                                 int32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

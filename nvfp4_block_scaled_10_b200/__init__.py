@@ -41,6 +41,9 @@ SIGNATURES = {
                           _vp, _vp]),
     "nvfp4_gemm_per_token": (_i32, [_vp, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64,
                                     _vp, _sz, _vp, _vp]),
+    "nvfp4_gemm_act_f32_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "nvfp4_gemm_act_f32": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _sz, _vp,
+                                  _vp]),
 }
 
 _lib = None
@@ -238,4 +241,32 @@ def nvfp4_gemm(a_q: torch.Tensor, a_sf: torch.Tensor, a_g: torch.Tensor, w_q: to
               _ptr(out), M, N, K, _ptr(workspace), 0 if workspace is None else workspace.numel(),
               _ptr(dev_status), _stream(stream)),
            "nvfp4_gemm_per_token" if per_token_a else "nvfp4_gemm")
+    return out
+
+
+def nvfp4_gemm_act_f32_workspace_bytes(M: int, N: int, K: int) -> int:
+    return lib().nvfp4_gemm_act_f32_workspace_bytes(M, N, K)
+
+
+def nvfp4_gemm_act_f32(a_q: torch.Tensor, a_sf32: torch.Tensor, w_q: torch.Tensor,
+                       w_sf: torch.Tensor, w_scale: torch.Tensor, out: torch.Tensor | None = None,
+                       dev_status: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[M, N] fp16 under the fp32 activation-scale contract: a_sf32 fp32 [M, K/16] (or
+    [M, 1, K/16]) combined activation scales, w_scale fp32 [1] multiplying the weight."""
+    M, K2 = a_q.shape
+    N = w_q.shape[0]
+    K = 2 * K2
+    if a_sf32.dtype != torch.float32 or a_sf32.numel() != M * (K // 16) or not a_sf32.is_contiguous():
+        raise ValueError("a_sf32 must be a contiguous fp32 tensor of M x K/16 scales")
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float16, device=a_q.device)
+    nbytes = nvfp4_gemm_act_f32_workspace_bytes(M, N, K)
+    if workspace is None and nbytes > 0:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=a_q.device)
+    _check(lib().nvfp4_gemm_act_f32(_ptr(a_q), _ptr(a_sf32), _ptr(w_q), _ptr(w_sf), _ptr(w_scale),
+                                    _ptr(out), M, N, K, _ptr(workspace),
+                                    0 if workspace is None else workspace.numel(),
+                                    _ptr(dev_status), _stream(stream)),
+           "nvfp4_gemm_act_f32")
     return out

@@ -239,4 +239,37 @@ int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int a_layout, 
                    workspace_bytes, dev_status, stream);
 }
 
+size_t nvfp4_gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  const DeviceInfo *d = device_info();
+  if (d == nullptr) return 0;
+  return gemm_act_f32_workspace_bytes(M, N, K, d->num_sms);
+}
+
+int nvfp4_gemm_act_f32(const uint8_t *a_q, const float *a_sf32, const uint8_t *w_q,
+                       const uint8_t *w_sf, const float *w_scale, void *out, int64_t M, int64_t N,
+                       int64_t K, void *workspace, size_t workspace_bytes, int32_t *dev_status,
+                       void *stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || N % 8 != 0) return NVFP4_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return NVFP4_OK;
+  if (a_q == nullptr || a_sf32 == nullptr || w_q == nullptr || w_sf == nullptr ||
+      w_scale == nullptr || out == nullptr)
+    return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(a_q) || !aligned16(a_sf32) || !aligned16(w_q) || !aligned16(w_sf) ||
+      !aligned16(out) || (reinterpret_cast<uintptr_t>(w_scale) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(dev_status) & 3u) != 0)
+    return NVFP4_ERR_MISALIGNED;
+  if (M > (int64_t(1) << 31) - 256 || N > (int64_t(1) << 31) - 256 || !gemm_act_f32_supported(K))
+    return NVFP4_ERR_UNSUPPORTED;
+  const DeviceInfo *d = device_info();
+  if (d == nullptr) return NVFP4_ERR_CUDA;
+  const size_t ws_need = gemm_act_f32_workspace_bytes(M, N, K, d->num_sms);
+  if (ws_need > 0 && (workspace == nullptr || workspace_bytes < ws_need)) return NVFP4_ERR_INVALID_ARG;
+  if (ws_need > 0 && !aligned16(workspace)) return NVFP4_ERR_MISALIGNED;
+  GemmArgs g{a_q,       nullptr,         NVFP4_SF_8x4, nullptr, w_q, w_sf,
+             nullptr,   out,             M,            N,       K,   dev_status,
+             workspace, workspace_bytes, 0,            a_sf32,  w_scale};
+  return finish(launch_gemm_act_f32(g, d->num_sms, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -486,12 +486,17 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
 constexpr int kDecBN = 32;
 constexpr int kDecMaxSfbBytes = 48 * 1024;  // preloaded activation scales: K <= 24576
 
-template <int STAGES>
+// NPL = 1: E4M3 activation scales. NPL = 3: fp32 activation scales split per row into three
+// planes of E4M3 codes (see split_act_scales). The MMA's N operand then holds the 32 token
+// rows three times (rows 32 p + j = token j under plane p's scales), one N = 96 MMA per K step
+// makes three partial sums per token, and the epilogue adds them.
+template <int STAGES, int NPL = 1>
 struct DecCfg {
+  static constexpr int kMmaN = kDecBN * NPL;
   static constexpr int kABytes = kBM * kBKBytes;                 // 16 KB of weights
-  static constexpr int kBBytes = kDecBN * kBKBytes;              // 4 KB of activations
+  static constexpr int kBBytes = kMmaN * kBKBytes;               // 4 KB of activations a copy
   static constexpr int kSfaBytes = kK64PerStage * kSfAtomBytes;  // 2 KB of weight scales
-  static constexpr int kSfbBytes = kK64PerStage * kSfAtomBytes;  // 2 KB of activation atoms
+  static constexpr int kSfbBytes = NPL > 1 ? 0 : kK64PerStage * kSfAtomBytes;  // 128x4 atoms
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
   static constexpr int kOffSfa = kOffB + STAGES * kBBytes;
@@ -501,18 +506,22 @@ struct DecCfg {
   // full[S], empty[S], sf_full[S], acc_full[2], acc_empty[2], sfb_ready, tmem slot + flag
   static constexpr int kBarBytes = (3 * STAGES + 2 * kAccBufs + 1) * 8 + 16;
   static constexpr int kOffSfb = (kOffBar + kBarBytes + 127) / 128 * 128;  // 8x4 rows 0..31
-  static constexpr int kAccCols = kDecBN;
-  static constexpr int kSlotCols = kK64PerStage * (4 + 4);  // A scales 4 columns, B 4 (1 used)
+  static constexpr int kAccCols = kMmaN;
+  // per K step: A scales 4 columns, B scales 4 (column p for the rows of plane p)
+  static constexpr int kSlotCols = kK64PerStage * (4 + 4);
   static constexpr int kSfCol0 = kAccBufs * kAccCols;
   static constexpr int kTmemCols = 512;
   static constexpr int kEpiWarps = 4;
   static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
   static_assert(kSfCol0 + STAGES * kSlotCols <= kTmemCols, "TMEM columns");
-  // the 8x4 copy holds 4 blocks of K/64 x 32 bytes
+  // E4M3 scales: the 8x4 copy of 4 blocks of K/64 x 32 bytes. fp32 scales: 2 x 32 fp32 row
+  // factors, then the plane words of two K steps' stages, [2][kK64PerStage][NPL][32] words.
+  static constexpr int kOffXbuf = 256;
   static constexpr int smem_bytes(int k64_total, bool sfb_8x4) {
-    return kOffSfb + (sfb_8x4 ? k64_total * 128 : 0) + 1024;
+    return kOffSfb + (NPL == 1 ? (sfb_8x4 ? k64_total * 128 : 0) : kOffXbuf + 2 * kK64PerStage * NPL * 128) +
+           1024;
   }
-  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(kDecBN >> 3) << 17) |
+  static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(kMmaN >> 3) << 17) |
                                      (uint32_t(kBM >> 4) << 24);
 };
 
@@ -531,6 +540,8 @@ struct DecParams {
   float *partials;      // [tiles][max_pieces][128][32] fp32
   int *counters;        // [tiles], zero on entry
   int32_t *dev_status;
+  const float *a_sf32;  // NPL = 3: fp32 activation scales [M, K/16]
+  const float *w_scale; // NPL = 3: fp32 weight dequantization scale (multiplies)
 };
 
 // Contiguous unit range [u0, u1) of CTA c among G over U units (units = tile x K-step).
@@ -544,29 +555,113 @@ __device__ __forceinline__ int dec_owner(int64_t u, int G, int64_t U) {
   return static_cast<int>(((u + 1) * G - 1) / U);
 }
 
-// AND of `v` over the `nthreads` threads of named barrier 1 (the epilogue warps).
-__device__ __forceinline__ bool epi_all(bool v, int nthreads) {
+// AND of `v` over the `nthreads` threads of named barrier `id` (a group of warps that must
+// leave a loop together).
+__device__ __forceinline__ bool group_all(bool v, int id, int nthreads) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred pi, po;\n\t"
       "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, 1, %2, pi;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
       "selp.u32 %0, 1, 0, po;\n\t}"
       : "=r"(r)
-      : "r"(static_cast<uint32_t>(v)), "r"(nthreads)
+      : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(nthreads)
       : "memory");
   return r != 0;
 }
+
+// Named barrier 1: the epilogue warps; 2: the scale warps.
+__device__ __forceinline__ bool epi_all(bool v, int nthreads) { return group_all(v, 1, nthreads); }
 
 __device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t v) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
 
-template <int STAGES>
-__global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
+// The largest E4M3 value <= t, for 0 <= t <= 448 (as an fp32 value). Every E4M3 value is
+// k * 2^E with an integer 0 <= k <= 15, so cutting t to four significant bits (normal range,
+// t >= 2^-6) or to a multiple of 2^-9 (subnormal range) lands on one, and t minus it is exact.
+__device__ __forceinline__ float e4m3_floor(float t) {
+  if (t >= 0x1p-6f) return __uint_as_float(__float_as_uint(t) & 0xFFF00000u);
+  return __fmul_rn(floorf(__fmul_rn(t, 512.0f)), 0x1p-9f);
+}
+
+// fp32 activation scales ("Fused Nvfp4 GEMM All Reduce Plugin": a combined FP32 scale
+// [B,1,K/16] per activation block, which the block-scaled MMA cannot take) become NPL planes of
+// E4M3 codes and one fp32 factor per row: with rho = max_c sa[r,c] / 448 and t = sa * (448 /
+// max) <= 448, plane 1 holds floor_E4M3(t), plane 2 floor_E4M3 of the exact remainder, plane 3
+// the remainder rounded to nearest. Each floor keeps at least four significant bits, so
+// rho * (v1 + v2 + v3) is within 2^-12 of sa relative (blocks below 2^-6 / 448 of the row
+// maximum within 2^-10 * rho absolute), and all codes are non-negative, as the MMA's unsigned
+// scales need. A negative, NaN or infinite scale is an argument error: its block counts as
+// zero and kDevErrBadScale is ORed into the status word.
+//
+// Row factors: warp q finds the maxima of rows 8q .. 8q+7 (the loads of all eight rows in
+// flight together) and stores 448 / max and alpha = rho * w_scale per row (zero past M).
+__device__ void act_scale_row_factors(const DecParams &p, int q, int lane, float *inv_s,
+                                      float *alpha_s, int64_t k64_per_row) {
+  constexpr int kRows = 8;
+  const int groups = static_cast<int>(k64_per_row);  // 4-column groups per row (K / 64)
+  const int r0 = q * kRows;
+  const float4 *src[kRows];
+  bool live[kRows];
+#pragma unroll
+  for (int i = 0; i < kRows; ++i) {
+    live[i] = r0 + i < p.M;
+    src[i] = reinterpret_cast<const float4 *>(p.a_sf32 + (live[i] ? r0 + i : 0) * (k64_per_row * 4));
+  }
+  float mx[kRows];
+#pragma unroll
+  for (int i = 0; i < kRows; ++i) mx[i] = 0.0f;
+  for (int g = lane; g < groups; g += 32) {
+    float4 v[kRows];
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) v[i] = live[i] ? __ldg(src[i] + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < kRows; ++i) {
+      const float e[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (e[j] >= 0.0f && e[j] <= FLT_MAX) mx[i] = fmaxf(mx[i], e[j]);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kRows; ++i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
+    if (lane == 0) {
+      const bool use = live[i] && mx[i] > 0.0f;
+      inv_s[r0 + i] = use ? __fdiv_rn(448.0f, mx[i]) : 0.0f;
+      alpha_s[r0 + i] = use ? __fmul_rn(__fdiv_rn(mx[i], 448.0f), p.w_scale[0]) : 0.0f;
+    }
+  }
+}
+
+// The NPL plane words (four E4M3 codes each, one K64 step of one row) of four fp32 scales.
+template <int NPL>
+__device__ __forceinline__ void split_scale_word(float4 v, float inv, uint32_t (&w)[NPL], bool &bad) {
+  const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int pl = 0; pl < NPL; ++pl) w[pl] = 0u;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const bool ok = e[j] >= 0.0f && e[j] <= FLT_MAX;
+    bad |= !ok;
+    float t = ok ? fminf(__fmul_rn(e[j], inv), 448.0f) : 0.0f;
+#pragma unroll
+    for (int pl = 0; pl + 1 < NPL; ++pl) {
+      const float f = e4m3_floor(t);
+      w[pl] |= cvt_e4m3(f) << (8 * j);
+      t = __fsub_rn(t, f);
+    }
+    w[NPL - 1] |= cvt_e4m3(t) << (8 * j);
+  }
+}
+
+template <int STAGES, int NPL>
+__global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     gemm_nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
                              const __grid_constant__ CUtensorMap tmap_a, const DecParams p) {
-  using C = DecCfg<STAGES>;
+  using C = DecCfg<STAGES, NPL>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -585,6 +680,8 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
   const int num_k64 = static_cast<int>(p.K / 64);
   const int num_kt = (num_k64 + kK64PerStage - 1) / kK64PerStage;
   const int64_t k64_per_row = p.K / 64;
+  float *inv_s = reinterpret_cast<float *>(smem + C::kOffSfb);  // fp32 scales: 448 / row max
+  float *alpha_s = inv_s + kDecBN;                                // and rho * w_scale
   const int64_t U = static_cast<int64_t>(p.tiles) * num_kt;
   const int G = gridDim.x;
   const int c = blockIdx.x;
@@ -601,7 +698,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], C::kEpiWarps);
     }
-    mbar_init(sfb_ready, 1);
+    mbar_init(sfb_ready, NPL > 1 ? 4 : 1);  // the bulk copy, or the four scale warps' split
     fence_mbar_init();
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_a);
@@ -617,7 +714,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (p.a_sf_8x4 && lane == 0) {
+    if (NPL == 1 && p.a_sf_8x4 && lane == 0) {
       // rows 0..31 of the 8x4 activation scales: four blocks of K/64 x 32 contiguous bytes
       const uint32_t blk = static_cast<uint32_t>(k64_per_row * 32);
       const int nblk = static_cast<int>(p.a_sf_rows / 8);
@@ -647,7 +744,10 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + sf_bytes);
           tma_load_2d(smem + C::kOffA + stage * C::kABytes, &tmap_w, kt * kBKBytes,
                       static_cast<int32_t>(w0), &full[stage]);
-          tma_load_2d(smem + C::kOffB + stage * C::kBBytes, &tmap_a, kt * kBKBytes, 0, &full[stage]);
+#pragma unroll
+          for (int pl = 0; pl < NPL; ++pl)  // the token tile once per scale plane
+            tma_load_2d(smem + C::kOffB + stage * C::kBBytes + pl * (kDecBN * kBKBytes), &tmap_a,
+                        kt * kBKBytes, 0, &full[stage]);
           bulk_g2s(smem + C::kOffSfa + stage * C::kSfaBytes,
                    p.w_sf + ((w0 / 128) * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
                    &full[stage]);
@@ -721,12 +821,35 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t it = 0;
     bool ok = true;
+    if constexpr (NPL > 1) {
+      act_scale_row_factors(p, q, lane, inv_s, alpha_s, k64_per_row);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sfb_ready);
+    }
     if (p.a_sf_8x4 && !mbar_wait_warp(sfb_ready, 0, kWaitTimeoutNs)) {
       if (lane == 0) report_timeout(p.dev_status);
       ok = false;
     }
+    if constexpr (NPL > 1) ok = group_all(ok, 2, 128);  // the scale warps enter the loop together
     // token `lane`'s 8x4 words: block lane / 8, byte (lane % 8) * 4 of each 32-byte step
     const uint8_t *my8x4 = sfb_8x4 + (lane / 8) * (k64_per_row * 32) + (lane % 8) * 4;
+    // fp32 scales: token `lane`'s row and factor (a token past M reads row 0 with factor 0)
+    const float4 *my_sf32 = nullptr;
+    float my_inv = 0.0f;
+    bool bad = false;
+    if constexpr (NPL > 1) {
+      my_sf32 = reinterpret_cast<const float4 *>(p.a_sf32 + (lane < p.M ? lane : 0) * (k64_per_row * 4));
+      my_inv = ok ? inv_s[lane] : 0.0f;
+    }
+    // warp q splits K64 step q of each stage (token `lane`'s four fp32 scales, loaded one
+    // stage ahead) and the four warps exchange the plane words through shared memory
+    float4 pre = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto load_step = [&](int ktn) {
+      const int k64 = ktn * kK64PerStage + q;
+      pre = (ktn >= 0 && k64 < num_k64) ? __ldg(my_sf32 + k64) : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    uint32_t *xbuf = reinterpret_cast<uint32_t *>(smem + C::kOffSfb + C::kOffXbuf);
+    if constexpr (NPL > 1) load_step(static_cast<int>(u0 % num_kt));
     for (int64_t u = u0; u < u1 && ok;) {
       const int tile = static_cast<int>(u / num_kt);
       const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
@@ -734,14 +857,29 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
       for (int kt = kb; kt < ke; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
-        if (!mbar_wait_warp(&full[stage], round & 1, kWaitTimeoutNs)) {
+        const int k64_0 = kt * kK64PerStage;
+        const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+        // fp32 scales: split this stage's words before the wait (they need no stage data),
+        // the next stage's scales loading meanwhile (the next segment starts a tile at K = 0)
+        uint32_t *xb = xbuf + (it & 1) * (kK64PerStage * NPL * 32);
+        if constexpr (NPL > 1) {
+          const float4 cur = pre;
+          load_step(kt + 1 < ke ? kt + 1 : (u + (ke - kb) < u1 ? 0 : -1));
+          uint32_t w[NPL];
+          split_scale_word<NPL>(cur, my_inv, w, bad);
+#pragma unroll
+          for (int pl = 0; pl < NPL; ++pl) xb[(q * NPL + pl) * 32 + lane] = w[pl];
+        }
+        bool got = mbar_wait_warp(&full[stage], round & 1, kWaitTimeoutNs);
+        // the four scale warps agree (and publish their words) before any leaves or reads:
+        // a buffer is rewritten two stages later, after every warp passed the next agreement
+        if constexpr (NPL > 1) got = group_all(got, 2, 128);
+        if (!got) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
           break;
         }
         tc_fence_after();
-        const int k64_0 = kt * kK64PerStage;
-        const int nk64 = min(kK64PerStage, num_k64 - k64_0);
         const uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
         const uint32_t slot = lane_base + C::kSfCol0 + stage * C::kSlotCols;
         // A (weights): row 32 q + lane's word at column (step base + q); B (tokens, N = 32):
@@ -750,11 +888,18 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
           const uint32_t wa =
               *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
           tmem_st_x4_rep(slot + a * 4, wa);
-          const uint32_t wb =
-              p.a_sf_8x4 ? *reinterpret_cast<const uint32_t *>(my8x4 + (k64_0 + a) * 32)
-                         : *reinterpret_cast<const uint32_t *>(
-                               smem + C::kOffSfbStage + stage * C::kSfbBytes + a * kSfAtomBytes + lane * 16);
-          tmem_st_x1(slot + kK64PerStage * 4 + a * 4, wb);
+          if constexpr (NPL > 1) {
+#pragma unroll
+            for (int pl = 0; pl < NPL; ++pl)
+              tmem_st_x1(slot + kK64PerStage * 4 + a * 4 + pl, xb[(a * NPL + pl) * 32 + lane]);
+          } else if (p.a_sf_8x4) {
+            tmem_st_x1(slot + kK64PerStage * 4 + a * 4,
+                       *reinterpret_cast<const uint32_t *>(my8x4 + (k64_0 + a) * 32));
+          } else {
+            tmem_st_x1(slot + kK64PerStage * 4 + a * 4,
+                       *reinterpret_cast<const uint32_t *>(smem + C::kOffSfbStage + stage * C::kSfbBytes +
+                                                           a * kSfAtomBytes + lane * 16));
+          }
         }
         tmem_wait_st();
         tc_fence_before();
@@ -763,13 +908,22 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
       }
       u += ke - kb;
     }
+    if (bad && p.dev_status != nullptr) atomicOr(p.dev_status, kDevErrBadScale);
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;  // weight row within the tile (accumulator lane)
     float alpha[kDecBN];  // per token (accumulator column)
+    if constexpr (NPL > 1) {
+      // the row factors come from the scale warps (zero if they never arrived: the
+      // accumulator waits below then give up too)
+      const bool got = mbar_wait_warp(sfb_ready, 0, kWaitTimeoutNs);
 #pragma unroll
-    for (int j = 0; j < kDecBN; ++j) alpha[j] = out_alpha(p.ga, p.ga_per_row, p.gw, j, p.M);
+      for (int j = 0; j < kDecBN; ++j) alpha[j] = got ? alpha_s[j] : 0.0f;
+    } else {
+#pragma unroll
+      for (int j = 0; j < kDecBN; ++j) alpha[j] = out_alpha(p.ga, p.ga_per_row, p.gw, j, p.M);
+    }
     uint32_t seg = 0;
     for (int64_t u = u0; u < u1; ++seg) {
       const int tile = static_cast<int>(u / num_kt);
@@ -794,6 +948,18 @@ __global__ void __launch_bounds__(DecCfg<STAGES>::kThreads, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 8; ++j) vals[cc + j] = __uint_as_float(v[j]);
+      }
+      // the planes' partial sums of token j sit in columns j, 32 + j, 64 + j
+#pragma unroll
+      for (int pl = 1; pl < NPL; ++pl) {
+#pragma unroll
+        for (int cc = 0; cc < kDecBN; cc += 8) {
+          uint32_t v[8];
+          tmem_ld_32x32b_x8(t_acc + pl * kDecBN + cc, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) vals[cc + j] = __fadd_rn(vals[cc + j], __uint_as_float(v[j]));
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -1389,9 +1555,9 @@ struct DecPlan {
   bool usable = false;
 };
 
-static DecPlan dec_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
+static DecPlan dec_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool sfb_fits = true) {
   DecPlan d;
-  if (M > kDecBN || K / 64 * 128 > kDecMaxSfbBytes) return d;
+  if (M > kDecBN || !sfb_fits) return d;
   const int64_t num_kt = (K / 64 + kK64PerStage - 1) / kK64PerStage;
   d.tiles = static_cast<int>((N + kBM - 1) / kBM);
   const int64_t U = d.tiles * num_kt;
@@ -1407,14 +1573,21 @@ static DecPlan dec_plan(int64_t M, int64_t N, int64_t K, int num_sms) {
   return d;
 }
 
+static bool sfb_8x4_fits(int64_t K) { return K / 64 * 128 <= kDecMaxSfbBytes; }
+
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
-  const DecPlan d = dec_plan(M, N, K, num_sms);
+  const DecPlan d = dec_plan(M, N, K, num_sms, sfb_8x4_fits(K));
   return d.usable ? d.partial_bytes + d.counter_bytes : 0;
 }
 
-template <int STAGES>
+size_t gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
+  const DecPlan d = dec_plan(M < kDecBN ? M : kDecBN, N, K, num_sms);
+  return d.usable ? d.partial_bytes + d.counter_bytes : 0;
+}
+
+template <int STAGES, int NPL = 1>
 static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t st) {
-  using C = DecCfg<STAGES>;
+  using C = DecCfg<STAGES, NPL>;
   CUtensorMap mw, ma;
   const int64_t kb = g.K / 2;
   if (!make_operand_map(&mw, g.w_q, g.N, kb, kBM)) return cudaErrorInvalidValue;
@@ -1422,8 +1595,10 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   DecParams p{};
   p.w_sf = g.w_sf;
   p.a_sf = g.a_sf;
-  p.a_sf_8x4 = g.a_layout == kSf8x4 ? 1 : 0;
-  p.a_sf_rows = p.a_sf_8x4 ? (g.M + 7) / 8 * 8 : (g.M + 127) / 128 * 128;
+  p.a_sf_8x4 = (NPL > 1 || g.a_layout == kSf8x4) ? 1 : 0;
+  p.a_sf_rows = NPL > 1 ? kDecBN : p.a_sf_8x4 ? (g.M + 7) / 8 * 8 : (g.M + 127) / 128 * 128;
+  p.a_sf32 = g.a_sf32;
+  p.w_scale = g.w_scale;
   p.ga = g.a_g;
   p.gw = g.w_g;
   p.ga_per_row = g.a_g_per_row;
@@ -1439,15 +1614,35 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   cudaError_t e = cudaMemsetAsync(p.counters, 0, d.counter_bytes, st);
   if (e != cudaSuccess) return e;
   const int smem = C::smem_bytes(static_cast<int>(g.K / 64), p.a_sf_8x4 != 0);
-  e = ensure_smem_attr(gemm_nvfp4_decode_kernel<STAGES>, smem);
+  e = ensure_smem_attr(gemm_nvfp4_decode_kernel<STAGES, NPL>, smem);
   if (e != cudaSuccess) return e;
-  gemm_nvfp4_decode_kernel<STAGES><<<d.grid, C::kThreads, smem, st>>>(mw, ma, p);
+  gemm_nvfp4_decode_kernel<STAGES, NPL><<<d.grid, C::kThreads, smem, st>>>(mw, ma, p);
   return cudaGetLastError();
+}
+
+bool gemm_act_f32_supported(int64_t K) { return K / 2 <= (int64_t(1) << 31); }
+
+// The GEMM with fp32 activation scales: the small-M stream-K kernel with three scale planes,
+// once per 32 activation rows (the rows of a chunk are independent; the chunks run in stream
+// order and share the workspace).
+cudaError_t launch_gemm_act_f32(const GemmArgs &g, int num_sms, cudaStream_t st) {
+  for (int64_t m0 = 0; m0 < g.M; m0 += kDecBN) {
+    GemmArgs c = g;
+    c.M = g.M - m0 < kDecBN ? g.M - m0 : kDecBN;
+    c.a_q = g.a_q + m0 * (g.K / 2);
+    c.a_sf32 = g.a_sf32 + m0 * (g.K / 16);
+    c.out = static_cast<__half *>(g.out) + m0 * g.N;
+    const DecPlan d = dec_plan(c.M, g.N, g.K, num_sms);
+    if (!d.usable) return cudaErrorNotSupported;
+    const cudaError_t e = run_decode<7, 3>(c, d, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_gemm(const GemmArgs &g, int num_sms, cudaStream_t st) {
   if (g.M <= 32) {
-    const DecPlan d = dec_plan(g.M, g.N, g.K, num_sms);
+    const DecPlan d = dec_plan(g.M, g.N, g.K, num_sms, sfb_8x4_fits(g.K));
     if (d.usable) return run_decode<7>(g, d, st);
     return run<32, 6, true>(g, num_sms, st);
   }

@@ -15,6 +15,7 @@ constexpr int kInFp16 = 1;
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s without progress
 constexpr int kDevErrTimeout = 1;
+constexpr int kDevErrBadScale = 2;  // an fp32 activation scale was negative, NaN or infinite
 
 // quantize.cu
 int *device_error_symbol();
@@ -49,10 +50,16 @@ struct GemmArgs {
   void *workspace;
   size_t workspace_bytes;
   int a_g_per_row;  // a_g is [M]: one activation encode scale per row
+  const float *a_sf32 = nullptr;   // fp32 activation scales [M, K/16] (launch_gemm_act_f32)
+  const float *w_scale = nullptr;  // fp32 weight dequantization scale (launch_gemm_act_f32)
 };
 cudaError_t launch_gemm(const GemmArgs &args, int num_sms, cudaStream_t st);
 // Workspace the GEMM needs for (M, N, K) on a device with num_sms SMs (split-K partial sums
 // and tile counters of the small-M path; 0 otherwise).
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+// The GEMM with fp32 activation scales [M, K/16] and a multiplying fp32 weight scale.
+cudaError_t launch_gemm_act_f32(const GemmArgs &args, int num_sms, cudaStream_t st);
+size_t gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms);
+bool gemm_act_f32_supported(int64_t K);
 
 }  // namespace nvfp4

@@ -344,6 +344,27 @@ def gemm_loops(a_q, a_sf_lin, a_g, w_q, w_sf_lin, w_g, want_f64: bool = False):
     return (out16, out64) if want_f64 else out16
 
 
+def gemm_act_f32(a_q, a_sf32, w_q, w_sf_lin, w_scale, want_f64: bool = False):
+    """The GEMM under the activation contract of "Fused Nvfp4 GEMM All Reduce Plugin"
+    (TensorRT-Edge-LLM C++ API, inputs [1] activation_scale FP32 [B,1,K/16] and [4]
+    weight_f32_scale): the activation's block scales arrive as combined fp32 values, and the
+    weight's scalar fp32 scale multiplies, as a DequantizeLinear scale does:
+        D = fp16_rn( sum_k E2M1(a[m,k]) * sa32[m,k/16] * E2M1(w[n,k]) * E4M3(sw[n,k/16]) * w_scale ).
+    E2M1 values come from the dequantizer with unit scales (code 0x38 is 1.0); each product
+    is exact in fp64; the sum by numpy's matmul; one rounding to fp16.
+    a_q [M,K/2], a_sf32 fp32 [M,K/16] (or [M,1,K/16]), w_q [N,K/2], w_sf_lin [N,K/16]."""
+    qa = _c(a_q, np.uint8)
+    M, K2 = qa.shape
+    K = 2 * K2
+    s32 = np.asarray(a_sf32, dtype=np.float32).reshape(M, K // 16).astype(np.float64)
+    e2m1_a = dequantize(qa, np.full((M, K // 16), 0x38, np.uint8), 1.0)
+    da = e2m1_a * np.repeat(s32, 16, axis=1)
+    dw = dequantize(w_q, w_sf_lin, 1.0) * float(np.float32(w_scale))
+    out64 = np.matmul(da, dw.T)
+    out16 = f64_to_f16(out64.reshape(-1)).reshape(out64.shape)
+    return (out16, out64) if want_f64 else out16
+
+
 # ----------------------------------------------------------------------------- traffic
 
 def swiglu_quant_traffic_as_printed(N: int, H: int):

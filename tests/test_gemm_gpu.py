@@ -191,3 +191,115 @@ def test_per_token_quantize_then_gemm_pipeline():
     out = nv.nvfp4_gemm(aq_d, asf_d, ag_d, wq_d, wsf_d, gw_d, per_token_a=True)
     torch.cuda.synchronize()
     gemm_close(out.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+
+
+# ------------------------------------------------------------------ fp32 activation scales
+
+def _e4m3_f64(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+def _act_f32_scales(kind, M, K, seed):
+    rng = np.random.default_rng(seed)
+    if kind == "product":  # E4M3 block scale x fp32 dequantization scale, as DequantizeLinear
+        codes = rng.integers(0x10, 0x7F, (M, K // 16), dtype=np.uint8)
+        return np.float32(_e4m3_f64(codes) * np.float64(np.float32(1.0 / 37.0)))
+    if kind == "wide":  # every block its own binade over 2^-22 .. 2^2, some zeros (the
+        # largest kept small enough that the fp16 result stays finite)
+        s = np.float32(2.0 ** rng.uniform(-22, 1, (M, K // 16)) * rng.uniform(1, 2, (M, K // 16)))
+        s[rng.random(s.shape) < 0.05] = 0.0
+        return s
+    raise ValueError(kind)
+
+
+def _run_act_f32(nv, a, sa32, w, sw, w_scale):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = nv.nvfp4_gemm_act_f32(torch.from_numpy(a).cuda(),
+                                torch.from_numpy(np.ascontiguousarray(sa32)).cuda(),
+                                torch.from_numpy(w).cuda(),
+                                torch.from_numpy(orc.swizzle(sw, orc.L128x4)).cuda(),
+                                torch.tensor([w_scale], dtype=torch.float32, device="cuda"),
+                                dev_status=status)
+    torch.cuda.synchronize()
+    return out.cpu().view(torch.int16).numpy().view(np.uint16), status.item()
+
+
+# M <= 32 one launch; M > 32 one launch per 32 rows (ragged last chunk); K = 64 a single MMA
+# K step; K up to 32768 (the scales are split per pipeline stage, so K has no limit).
+ACT_F32 = [(1, 256, 512), (5, 136, 64), (32, 512, 1024), (33, 256, 512), (80, 1032, 2048),
+           (17, 1032, 8192), (8, 264, 16384), (2, 520, 32768)]
+
+
+@pytest.mark.parametrize("kind", ["product", "wide"])
+@pytest.mark.parametrize("M,N,K", ACT_F32)
+def test_gemm_act_f32_parity(M, N, K, kind):
+    nv = require_cuda()
+    seed = M * 31 + N + K
+    a = workloads.random_bytes((M, K // 2), seed)
+    w = workloads.random_bytes((N, K // 2), seed + 1)
+    sw = workloads.random_bytes((N, K // 16), seed + 3, 0x28, 0x48)
+    sa32 = _act_f32_scales(kind, M, K, seed + 2)
+    w_scale = float(np.float32(1.0 / 250.0))
+    _, ref = orc.gemm_act_f32(a, sa32, w, sw, w_scale, want_f64=True)
+    got, status = _run_act_f32(nv, a, sa32, w, sw, w_scale)
+    assert status == 0
+    gemm_close(got, ref)
+
+
+def test_gemm_act_f32_zero_rows_and_blocks():
+    """A row whose scales are all zero gives zeros (the split's row factor is then zero)."""
+    nv = require_cuda()
+    M, N, K = 6, 264, 1024
+    a = workloads.random_bytes((M, K // 2), 3)
+    w = workloads.random_bytes((N, K // 2), 4)
+    sw = workloads.random_bytes((N, K // 16), 5, 0x28, 0x48)
+    sa32 = _act_f32_scales("product", M, K, 6)
+    sa32[2] = 0.0
+    sa32[4, ::3] = 0.0
+    _, ref = orc.gemm_act_f32(a, sa32, w, sw, 0.5, want_f64=True)
+    got, status = _run_act_f32(nv, a, sa32, w, sw, 0.5)
+    assert status == 0
+    assert (got[2].view(np.float16) == 0).all()
+    gemm_close(got, ref)
+
+
+def test_gemm_act_f32_bad_scales_flagged():
+    """Negative, NaN and infinite activation scales are flagged in dev_status (value 2) and
+    their blocks count as zero; the rest of the result is unaffected."""
+    nv = require_cuda()
+    M, N, K = 4, 136, 512
+    a = workloads.random_bytes((M, K // 2), 13)
+    w = workloads.random_bytes((N, K // 2), 14)
+    sw = workloads.random_bytes((N, K // 16), 15, 0x28, 0x48)
+    sa32 = _act_f32_scales("product", M, K, 16)
+    bad = sa32.copy()
+    bad[0, 3] = -1.0
+    bad[1, 0] = np.nan
+    bad[3, 31] = np.inf
+    clean = sa32.copy()
+    clean[0, 3] = clean[1, 0] = clean[3, 31] = 0.0
+    _, ref = orc.gemm_act_f32(a, clean, w, sw, 1.0, want_f64=True)
+    got, status = _run_act_f32(nv, a, bad, w, sw, 1.0)
+    assert status == 2
+    gemm_close(got, ref)
+
+
+@pytest.mark.parametrize("M", [1, 32])
+def test_gemm_act_f32_decode_workload(decode_weights, M):
+    """The decode workload (W NVFP4 [28672, 8192]) under the fp32 activation contract: the
+    activation quantized by the oracle, its scales handed over as E4M3 value x fp32(1/ga) and
+    the weight scale as fp32(1/gw); 512 sampled output columns against the oracle."""
+    nv = require_cuda()
+    wq, ws, gw = decode_weights
+    a_bf16, _ = workloads.decode(M, N=16, K=8192)
+    ab = workloads.bits16(a_bf16)
+    ga = orc.global_scale(ab)
+    aq, sa, _ = orc.quantize(ab, g=ga)
+    sa32 = np.float32(_e4m3_f64(sa) * np.float64(np.float32(1.0 / ga)))
+    w_scale = float(np.float32(1.0 / gw))
+    cols = np.sort(np.random.default_rng(M + 5).choice(wq.shape[0], 512, replace=False))
+    _, ref = orc.gemm_act_f32(aq, sa32, wq[cols], ws[cols], w_scale, want_f64=True)
+    got, status = _run_act_f32(nv, aq, sa32, wq, ws, w_scale)
+    assert status == 0
+    gemm_close(got[:, cols], ref)

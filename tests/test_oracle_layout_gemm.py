@@ -217,3 +217,70 @@ def test_gemm_per_row_activation_scales(orc):
         _, loop_m = orc.gemm_loops(a[m:m + 1], sa[m:m + 1], float(g_rows[m]), w, sw, 2.0,
                                    want_f64=True)
         np.testing.assert_allclose(rows[m:m + 1], loop_m, rtol=1e-12, atol=1e-300)
+
+
+def _e4m3_values(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(
+        torch.float64).numpy()
+
+
+def test_gemm_act_f32_equals_scalar_contract_for_product_scales(orc):
+    """fp32 activation scales that are E4M3 scale / g exactly (g a power of two) and a weight
+    scale 1 / gw give the scalar-contract GEMM bit for bit: the two contracts name the same
+    real numbers then."""
+    rng = np.random.default_rng(21)
+    M, N, K = 5, 24, 128
+    a = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    w = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = rng.integers(0x08, 0x7F, (M, K // 16), dtype=np.uint8)
+    sw = rng.integers(0x20, 0x60, (N, K // 16), dtype=np.uint8)
+    ga, gw = 64.0, 0.25
+    sa32 = (_e4m3_values(sa) / ga).astype(np.float32)
+    assert np.array_equal(sa32.astype(np.float64) * ga, _e4m3_values(sa))  # exact
+    ref16, ref64 = orc.gemm(a, sa, ga, w, sw, gw, want_f64=True)
+    got16, got64 = orc.gemm_act_f32(a, sa32, w, sw, 1.0 / gw, want_f64=True)
+    np.testing.assert_array_equal(got64, ref64)
+    np.testing.assert_array_equal(got16, ref16)
+    # the [B,1,K/16] shape of the plugin reads the same
+    np.testing.assert_array_equal(orc.gemm_act_f32(a, sa32.reshape(M, 1, K // 16), w, sw, 4.0), ref16)
+
+
+def test_gemm_act_f32_brute_force_exact(orc):
+    """Against an exact rational sum (fractions) of the defining products, on a tiny case
+    with fp32 scales spread over many binades; the weight scale multiplies."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    M, N, K = 3, 4, 64
+    a = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    w = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sw = rng.integers(0x10, 0x70, (N, K // 16), dtype=np.uint8)
+    sa32 = np.float32(2.0 ** rng.uniform(-20, 20, (M, K // 16)) * rng.uniform(1, 2, (M, K // 16)))
+    w_scale = np.float32(0.0037)
+    e2m1 = lambda b: E2M1[b]  # noqa: E731
+    swv = _e4m3_values(sw)
+    got16, got64 = orc.gemm_act_f32(a, sa32, w, sw, w_scale, want_f64=True)
+    for m in range(M):
+        for n in range(N):
+            acc = Fraction(0)
+            for k in range(K):
+                av = e2m1((a[m, k // 2] >> (4 * (k % 2))) & 0xF)
+                wv = e2m1((w[n, k // 2] >> (4 * (k % 2))) & 0xF)
+                acc += (Fraction(float(av)) * Fraction(float(sa32[m, k // 16])) * Fraction(float(wv))
+                        * Fraction(float(swv[n, k // 16])) * Fraction(float(w_scale)))
+            exact = float(acc)
+            assert abs(got64[m, n] - exact) <= 1e-13 * max(abs(exact), 1e-300)
+            assert got16[m, n] == np.float16(exact).view(np.uint16)
+
+
+def test_gemm_act_f32_weight_scale_multiplies(orc):
+    rng = np.random.default_rng(8)
+    M, N, K = 2, 8, 64
+    a = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    w = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sw = rng.integers(0x20, 0x60, (N, K // 16), dtype=np.uint8)
+    sa32 = np.float32(rng.uniform(0.01, 3.0, (M, K // 16)))
+    _, one = orc.gemm_act_f32(a, sa32, w, sw, 1.0, want_f64=True)
+    _, three = orc.gemm_act_f32(a, sa32, w, sw, 3.0, want_f64=True)
+    _, eighth = orc.gemm_act_f32(a, sa32, w, sw, 0.125, want_f64=True)
+    np.testing.assert_allclose(three, 3.0 * one, rtol=1e-15, atol=0)
+    np.testing.assert_array_equal(eighth, one / 8.0)
