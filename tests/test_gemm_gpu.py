@@ -52,12 +52,14 @@ def _run(nv, ops, a_layout):
     return out.cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-# M <= 32: swap-AB tiles; 33..255: single-CTA 128 x 256 tiles; M >= 256: CTA-pair 256 x 256
-# tiles (ragged M, N and K tails, and more tiles than resident pairs so the accumulator is
-# reused).
+# M <= 32: swap-AB tiles; 33..255: single-CTA 128 x 256 tiles; M >= 256: CTA-pair tiles,
+# 256 x 256, or 256 x 384 where that needs fewer operand bytes per wave (4096 x 2560,
+# 2000 x 5000, 1536 x 4608, 2048 x 3072 on 148 SMs); ragged M, N and K tails, and more tiles
+# than resident pairs so the accumulator and the scale slots are reused.
 SMALL = [(1, 256, 512), (8, 256, 512), (16, 256, 512), (32, 512, 1024), (3, 136, 64),
          (33, 256, 512), (128, 256, 256), (130, 520, 320), (256, 1024, 2048), (300, 264, 4096),
-         (520, 776, 320), (4096, 2560, 512),
+         (520, 776, 320), (4096, 2560, 512), (2000, 5000, 320), (1536, 4608, 512),
+         (2048, 3072, 1024),
          (2, 20480, 1024), (32, 4096, 3072), (17, 1032, 8192)]
 
 
@@ -144,7 +146,7 @@ def test_gemm_prefill_workload():
 
 
 @pytest.mark.parametrize("M,N,K", [(8, 512, 1024), (32, 20480, 1024), (100, 520, 512),
-                                   (300, 264, 1024), (1024, 1024, 2048)])
+                                   (300, 264, 1024), (1024, 1024, 2048), (2048, 3072, 1024)])
 def test_gemm_per_token_activation_scales(M, N, K):
     """Activation quantized per token (one g per row, as nvfp4_quantize(per_token=True)
     writes), weights per tensor: nvfp4_gemm_per_token against the oracle GEMM with row
