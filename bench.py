@@ -1,7 +1,8 @@
 """Benchmark of the NVFP4 hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload per_token|swiglu|decode|prefill|tiny] [--m 32] [--a-layout 128x4|8x4]
+                    [--workload per_token|swiglu|swiglu_fp8|decode|decode_f32|prefill|tiny]
+                    [--m 32] [--a-layout 128x4|8x4] [--no-cpu-baseline] [--no-all-cores]
 
 Default workload: per-token NVFP4 quantize of X bf16 [8192, 7168] (N(0,1) with 0.1% of
 entries x50), one fp32 global scale per token, E4M3 scales in the 128x4 layout. A step is
@@ -11,7 +12,8 @@ copies that no step finds its input in the 126 MB L2.
 Prints one JSON line (rank 0). `value` is whole-job throughput in the workload's unit
 (GB/s of algorithmic bytes for the quantize kernels, TFLOP/s for the GEMMs), measured with
 CUDA events on the launching stream, max over ranks. Multi-GPU runs are independent
-replicas (weak scaling): the path has no exchange step.
+replicas (weak scaling): the path has no exchange step. `cpu_baseline` times the oracle on
+a bounded sample on one host core and, under `all_cores`, on every host core.
 """
 from __future__ import annotations
 
@@ -552,14 +554,60 @@ def _threads_used():
     return n
 
 
+def _oracle_rows(wl):
+    """The row-independent oracle workloads over all their rows: (run(lo, hi), rows, units
+    of the whole sample, desc). The oracle's C calls release the GIL, so threads over row slices run it
+    on all cores as it stands."""
+    import oracle
+    from nvfp4_block_scaled_10_b200 import workloads
+
+    if wl == "per_token":
+        bits = workloads.bits16(workloads.per_token(8192, 7168))
+        return (lambda lo, hi: oracle.quantize(bits[lo:hi], oracle.BF16, per_token=True)), 8192, \
+            algorithmic("per_token", M=8192, K=7168)["bytes"] / 1e9, "all 8192 rows"
+    if wl in ("swiglu", "swiglu_fp8"):
+        bits = workloads.bits16(workloads.swiglu(4096, 14336))
+        if wl == "swiglu":
+            run = lambda lo, hi: oracle.swiglu_quantize(bits[lo:hi], 2688.0 / 60.0, oracle.BF16)  # noqa: E731
+        else:
+            run = lambda lo, hi: oracle.swiglu_fp8(bits[lo:hi], 448.0 / 60.0, oracle.BF16)  # noqa: E731
+        return run, 4096, algorithmic(wl, M=4096, H=14336)["bytes"] / 1e9, "all 4096 rows"
+    return None
+
+
+def _all_cores(wl):
+    """The same oracle on every host core: row slices over one thread per core."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    spec = _oracle_rows(wl)
+    if spec is None:
+        return None
+    run, rows, units, desc = spec
+    n = max(1, min(os.cpu_count() or 1, rows))
+    cuts = [rows * i // n for i in range(n + 1)]
+    t = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=n) as ex:
+        list(ex.map(lambda i: run(cuts[i], cuts[i + 1]), range(n)))
+    dt = time.perf_counter() - t
+    return {"value": units / dt, "cores": n, "sample": desc, "seconds": dt}
+
+
 def cpu_baseline(wl, args):
+    import oracle
+
+    oracle.lib()  # build check and library load stay out of the timing
     fn, units, desc, unit = _oracle_sample(wl, args)
     t = time.perf_counter()
     fn()
     dt = time.perf_counter() - t
     cores = 1 if wl in ("per_token", "swiglu", "swiglu_fp8") else _threads_used()
-    return {"value": units / dt, "unit": unit, "cores": cores, "kind": "oracle",
-            "sample": desc, "seconds": dt}
+    out = {"value": units / dt, "unit": unit, "cores": cores, "kind": "oracle",
+           "sample": desc, "seconds": dt}
+    if not args.no_all_cores:
+        allc = _all_cores(wl)
+        if allc is not None:
+            out["all_cores"] = allc
+    return out
 
 
 def run_reference(args, rank, world):
@@ -598,6 +646,8 @@ def main():
     ap.add_argument("--m", type=int, default=32, help="tokens of the decode workload")
     ap.add_argument("--a-layout", default="128x4", choices=["128x4", "8x4"])
     ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--no-all-cores", action="store_true",
+                    help="skip the oracle timing on all host cores (cpu_baseline.all_cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time direct library calls instead of CUDA-graph replays of them")

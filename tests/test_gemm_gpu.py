@@ -305,3 +305,27 @@ def test_gemm_act_f32_decode_workload(decode_weights, M):
     got, status = _run_act_f32(nv, aq, sa32, wq, ws, w_scale)
     assert status == 0
     gemm_close(got[:, cols], ref)
+
+
+# ------------------------------------------------------------------ exact special case
+
+@pytest.mark.parametrize("M,N,K", [(8, 1032, 512), (100, 520, 512), (512, 1024, 512),
+                                   (2048, 3072, 512)])
+def test_gemm_bit_exact_when_accumulation_is_exact(M, N, K):
+    """With block scales in {1/2, 1, 2} and unit global scales every product is a multiple of
+    1/16 below 2^8, so every partial sum of K = 512 terms is exact in fp32 whatever the
+    accumulation order, and alpha = 1: the kernels' fp16 output must equal the oracle's single
+    rounding of the exact sum bit for bit. Shapes reach the decode (split-K), single-CTA and
+    both CTA-pair kernels."""
+    nv = require_cuda()
+    rng = np.random.default_rng(M + N)
+    a = workloads.random_bytes((M, K // 2), M + 1)
+    w = workloads.random_bytes((N, K // 2), N + 2)
+    codes = np.array([0x30, 0x38, 0x40], np.uint8)  # E4M3 0.5, 1, 2
+    sa = codes[rng.integers(0, 3, (M, K // 16))]
+    sw = codes[rng.integers(0, 3, (N, K // 16))]
+    ref = orc.gemm(a, sa, 1.0, w, sw, 1.0)
+    layouts = [orc.L128x4, orc.L8x4] if M <= 32 else [orc.L128x4]
+    for layout in layouts:
+        got = _run(nv, (a, sa, 1.0, w, sw, 1.0), layout)
+        assert np.array_equal(got, ref), f"{np.count_nonzero(got != ref)} outputs differ"
