@@ -182,6 +182,25 @@ def recorded_traffic(kernel_key):
     return e["bytes_per_launch"]
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(ms, dist, device):
+    """The largest of every rank's time (the job is as slow as its slowest rank); `ms` as is
+    with one rank. Every rank must call it, in the same order."""
+    if dist is None:
+        return ms
+    import torch
+
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.item()
+
+
+def job_throughput(world, units_per_rank_step, ms_per_step):
+    """Whole-job throughput: all ranks' units of one step over the slowest rank's step time."""
+    return world * units_per_rank_step / (ms_per_step / 1e3)
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, torch, dist):
@@ -358,12 +377,9 @@ def run_ours(args, rank, world, torch, dist):
         dist.barrier()
     total_ms = t0.elapsed_time(t1)
     launch_avg = total_ms / (args.steps * launches_per_step)
-    if dist is not None:
-        tt = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = tt.item()
+    total_ms = max_over_ranks(total_ms, dist, dev)
     ms_per_step = total_ms / args.steps
-    value = world * factor / (total_ms / 1e3 / args.steps)
+    value = job_throughput(world, factor, ms_per_step)
 
     # ---- end to end through the public API with host buffers (pinned), copies timed
     e2e = None
@@ -399,13 +415,9 @@ def run_ours(args, rank, world, torch, dist):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if dist is not None:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = tt.item()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
         d2h = h_q.numel() + (h_sf.numel() if h_sf is not None else 0) + (h_g.numel() * 4 if h_g is not None else 0)
-        e2e = {"value": world * factor / (e2e_ms / 1e3), "unit": unit,
+        e2e = {"value": job_throughput(world, factor, e2e_ms), "unit": unit,
                "h2d_bytes_per_step": h_in.numel() * 2, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms}
     elif wl in ("decode", "prefill", "tiny", "decode_f32"):
@@ -432,12 +444,8 @@ def run_ours(args, rank, world, torch, dist):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if dist is not None:
-            tt = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = tt.item()
-        e2e = {"value": world * factor / (e2e_ms / 1e3), "unit": unit,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, dist, dev)
+        e2e = {"value": job_throughput(world, factor, e2e_ms), "unit": unit,
                "h2d_bytes_per_step": sum(h.numel() for h in hs), "d2h_bytes_per_step": h_out.numel() * 2,
                "ms_per_step": e2e_ms}
 

@@ -365,6 +365,31 @@ def gemm_act_f32(a_q, a_sf32, w_q, w_sf_lin, w_scale, want_f64: bool = False):
     return (out16, out64) if want_f64 else out16
 
 
+def gemm_row_parallel(a_q, a_sf_lin, a_g, w_q, w_sf_lin, w_g, tp: int = 2,
+                      want_f64: bool = False):
+    """Row-parallel GEMM of "Fused Nvfp4 GEMM All Reduce Plugin" (TensorRT-Edge-LLM C++ API,
+    tp_size 2): K is split into tp equal shards; rank r's local output is the GEMM over its
+    shard rounded to fp16 (the plugin's rank-local FP16 [B,N]); the AllReduce sums the tp fp16
+    outputs (fp64 sum, one rounding to fp16 -- for two ranks the correctly rounded sum).
+    Returns fp16 bits [M,N], plus the fp64 sum of the unrounded partials when want_f64."""
+    qa, qw = _c(a_q, np.uint8), _c(w_q, np.uint8)
+    K = 2 * qa.shape[1]
+    assert K % (64 * tp) == 0, "each shard must hold whole 64-element MMA steps"
+    ks = K // tp
+    parts16, sum64 = [], 0.0
+    for r in range(tp):
+        b0, b1, c0, c1 = r * ks // 2, (r + 1) * ks // 2, r * ks // 16, (r + 1) * ks // 16
+        p16, p64 = gemm(qa[:, b0:b1], np.asarray(a_sf_lin)[:, c0:c1], a_g, qw[:, b0:b1],
+                        np.asarray(w_sf_lin)[:, c0:c1], w_g, want_f64=True)
+        parts16.append(p16.view(np.float16).astype(np.float64))
+        sum64 = sum64 + p64
+    total = parts16[0]
+    for p in parts16[1:]:
+        total = total + p
+    out16 = f64_to_f16(total.reshape(-1)).reshape(total.shape)
+    return (out16, sum64) if want_f64 else out16
+
+
 # ----------------------------------------------------------------------------- traffic
 
 def swiglu_quant_traffic_as_printed(N: int, H: int):

@@ -329,3 +329,57 @@ def test_gemm_bit_exact_when_accumulation_is_exact(M, N, K):
     for layout in layouts:
         got = _run(nv, (a, sa, 1.0, w, sw, 1.0), layout)
         assert np.array_equal(got, ref), f"{np.count_nonzero(got != ref)} outputs differ"
+
+
+# ------------------------------------------------------------------ row-parallel (tp) GEMM
+
+@pytest.mark.parametrize("M,N,K", [(8, 1032, 2048), (300, 520, 2048)])
+def test_row_parallel_shards_on_one_gpu(M, N, K):
+    """The two K shards' GEMMs (decode and single-CTA kernels) on one GPU, each against the
+    oracle's GEMM of that shard, and their fp16 sum (what the AllReduce computes) against the
+    oracle's row-parallel reading, within the two partials' tolerances plus one fp16 rounding.
+    No collective runs here."""
+    nv = require_cuda()
+    from nvfp4_block_scaled_10_b200 import tp
+    ops = _random_operands(M, N, K, seed=M + N + K + 7)
+    a, sa, ga, w, sw, gw = ops
+    d = _to_device(nv, *ops, orc.L128x4)
+    outs, bound = [], 0.0
+    for r in range(2):
+        out = nv.nvfp4_gemm(tp.shard_packed(d["a_q"], r, 2),
+                            tp.shard_scales(d["a_sf"], M, K, nv.SF_128x4, r, 2), d["a_g"],
+                            tp.shard_packed(d["w_q"], r, 2),
+                            tp.shard_scales(d["w_sf"], N, K, nv.SF_128x4, r, 2), d["w_g"])
+        k0, k1 = tp.k_shard_bounds(K, r, 2)
+        _, ref_r = orc.gemm(a[:, k0 // 2:k1 // 2], sa[:, k0 // 16:k1 // 16], ga,
+                            w[:, k0 // 2:k1 // 2], sw[:, k0 // 16:k1 // 16], gw, want_f64=True)
+        torch.cuda.synchronize()
+        gemm_close(out.cpu().view(torch.int16).numpy().view(np.uint16), ref_r)
+        outs.append(out)
+        bound = bound + 1e-3 * np.abs(ref_r) + 1e-3 * np.sqrt(np.mean(ref_r ** 2))
+    got = (outs[0] + outs[1]).cpu().view(torch.int16).numpy().view(np.uint16)
+    want = orc.gemm_row_parallel(*ops, tp=2).view(np.float16).astype(np.float64)
+    diff = np.abs(got.view(np.float16).astype(np.float64) - want)
+    assert np.all(diff <= bound + 2.0 ** -11 * np.abs(want))
+
+
+def test_row_parallel_nccl_one_rank():
+    """The row-parallel call through NCCL with a single rank equals the plain GEMM."""
+    nv = require_cuda()
+    import socket
+
+    import torch.distributed as dist
+
+    from nvfp4_block_scaled_10_b200 import tp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        d = _to_device(nv, *_random_operands(8, 520, 1024, seed=91), orc.L128x4)
+        ref = nv.nvfp4_gemm(**d)
+        got = tp.row_parallel_gemm(**d)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref)
+    finally:
+        dist.destroy_process_group()

@@ -284,3 +284,28 @@ def test_gemm_act_f32_weight_scale_multiplies(orc):
     _, eighth = orc.gemm_act_f32(a, sa32, w, sw, 0.125, want_f64=True)
     np.testing.assert_allclose(three, 3.0 * one, rtol=1e-15, atol=0)
     np.testing.assert_array_equal(eighth, one / 8.0)
+
+
+def test_gemm_row_parallel_reading(orc):
+    """tp = 1 is the GEMM itself; for tp = 2 and 4 the unrounded shard sums add up to the
+    full GEMM's fp64 sum (the shards partition K exactly) and the result is the full GEMM's
+    value to within the extra fp16 roundings of the partials."""
+    rng = np.random.default_rng(40)
+    M, N, K = 5, 24, 512
+    a = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    w = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    sa = rng.integers(0x28, 0x48, (M, K // 16), dtype=np.uint8)
+    sw = rng.integers(0x28, 0x48, (N, K // 16), dtype=np.uint8)
+    full16, full64 = orc.gemm(a, sa, 2.0, w, sw, 30.0, want_f64=True)
+    one16, one64 = orc.gemm_row_parallel(a, sa, 2.0, w, sw, 30.0, tp=1, want_f64=True)
+    np.testing.assert_array_equal(one16, full16)
+    np.testing.assert_array_equal(one64, full64)
+    for t in (2, 4):
+        o16, o64 = orc.gemm_row_parallel(a, sa, 2.0, w, sw, 30.0, tp=t, want_f64=True)
+        np.testing.assert_allclose(o64, full64, rtol=1e-12, atol=1e-12 * np.abs(full64).max())
+        got = o16.view(np.float16).astype(np.float64)
+        # t partial roundings and one final rounding, each at most half an fp16 ulp
+        bound = (t + 1) * 2.0 ** -11 * (np.abs(full64) + np.abs(full64).max() * 2.0 ** -4)
+        assert np.all(np.abs(got - full64) <= bound)
+    with pytest.raises(AssertionError):
+        orc.gemm_row_parallel(a[:, :96], sa[:, :12], 2.0, w[:, :96], sw[:, :12], 30.0, tp=2)
