@@ -108,3 +108,28 @@ def test_global_scale_and_swizzle_argument_checks(L):
     assert L.nvfp4_global_scale(P16, 0, 4, 32, 32, None, P16, 64, None) == nv.ERR_INVALID_ARG
     assert L.nvfp4_sf_swizzle(P16, P16, 4, 4, 5, None) == nv.ERR_INVALID_ARG
     assert L.nvfp4_sf_unswizzle(P16, P16, 0, 4, 1, None) == nv.OK
+
+
+def test_swiglu_fp8_argument_checks(L):
+    f = L.swiglu_fp8_quantize
+    assert f(P16, 0, 4, 24, 48, P16, P16, None) == nv.ERR_INVALID_ARG    # H % 16
+    assert f(P16, 0, 4, 32, 48, P16, P16, None) == nv.ERR_INVALID_ARG    # ldx < 2H
+    assert f(P16, 2, 4, 32, 64, P16, P16, None) == nv.ERR_INVALID_ARG    # dtype
+    assert f(P_ODD, 0, 4, 32, 64, P16, P16, None) == nv.ERR_MISALIGNED   # x
+    assert f(P16, 0, 4, 32, 64, None, P16, None) == nv.ERR_INVALID_ARG   # scale
+    assert f(P16, 0, 4, 32, 64, P16, P_ODD, None) == nv.ERR_MISALIGNED   # q
+    assert f(P16, 0, 0, 32, 64, None, None, None) == nv.OK               # empty
+
+
+def test_gemm_act_f32_argument_checks(L):
+    g = L.nvfp4_gemm_act_f32
+    a = (P16, P16, P16, P16, P16, P16)  # a_q, a_sf32, w_q, w_sf, w_scale, out
+    assert g(*a, 16, 256, 96, None, 0, None, None) == nv.ERR_INVALID_ARG      # K % 64
+    assert g(*a, 16, 250, 512, None, 0, None, None) == nv.ERR_INVALID_ARG     # N % 8
+    assert g(P16, None, P16, P16, P16, P16, 16, 256, 512, None, 0, None, None) == \
+        nv.ERR_INVALID_ARG                                                     # a_sf32
+    assert g(P16, P_ODD, P16, P16, P16, P16, 16, 256, 512, None, 0, None, None) == \
+        nv.ERR_MISALIGNED                                                      # a_sf32
+    assert g(P16, P16, P16, P16, ctypes.c_void_p(0x10002), P16, 16, 256, 512, None, 0, None,
+             None) == nv.ERR_MISALIGNED                                        # w_scale
+    assert g(*a, 0, 256, 512, None, 0, None, None) == nv.OK                    # empty
