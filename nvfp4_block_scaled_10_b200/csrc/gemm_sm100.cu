@@ -1640,10 +1640,9 @@ static cudaError_t run_pair(const GemmArgs &g, cudaStream_t st) {
 
 // Pair tile width by the operand bytes a CTA pair stages per wave: a 256 x BN tile stages
 // (256 + BN) rows of K, and the tiles run in waves over the resident pairs, so the bytes go as
-// waves x (256 + BN). The 384 tile's two tensor-memory scale slots put a cross-CTA round trip
-// (MMA commit, the peer's scale writes, its arrive on the leader) into every ring stage, which
-// eats most of its 13% byte saving: on B200 it measured 2% faster at 8192^3 and 1% slower at
-// 4096 x 4096 x 8192. It is taken only where the model gives it 10% or more.
+// waves x (256 + BN). The 384 tile's 13% byte saving mostly does not show up as time: on B200
+// it measured 2% faster at 8192^3 and 1% slower at 4096 x 4096 x 8192, with the scale-slot
+// ring ruled out as the cause. It is taken only where the model gives it 10% or more.
 static int pair_tile_width(int64_t M, int64_t N, int resident256, int resident384) {
   if (resident256 <= 0 || resident384 <= 0) return 256;
   const int64_t ta = (M + 255) / 256;
