@@ -1085,8 +1085,10 @@ struct PairCfg {
   static constexpr int kSlotCols = kSlotB2 + kK64PerStage * kSfb2ColsPerK64;
   static constexpr int kSfCol0 = kAccCols;
   static constexpr int kTmemCols = 512;
-  static constexpr int kEpiWarps = 8;
-  static constexpr int kColsPerEpiWarp = kN * 4 / kEpiWarps;  // 128 or 192
+  // epilogue: three warps per lane quarter for N = 384, two for 256: 128 columns each, so
+  // every warp holds its whole share in registers before it releases the accumulator
+  static constexpr int kEpiWarps = BN / 32;
+  static constexpr int kColsPerEpiWarp = kN * 4 / kEpiWarps;  // 128
   static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
   static_assert(BN == 256 || BN == 384, "pair tile width");
   static_assert(kSfCol0 + kSlots * kSlotCols <= kTmemCols, "TMEM columns");
@@ -1354,69 +1356,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col0;
       const int64_t m = m0 + C::kHalf * rank + row;
       __half *dst = p.out + m * p.N + n0 + col0;
-      if constexpr (BN == 256) {
-        // all 128 columns into registers, release the accumulator, then store
-        uint32_t h2[C::kColsPerEpiWarp / 2];
+      // all 128 columns into registers, release the accumulator, then store
+      uint32_t h2[C::kColsPerEpiWarp / 2];
 #pragma unroll
-        for (int c = 0; c < C::kColsPerEpiWarp; c += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(t_acc + c, v);
-          tmem_wait_ld();
+      for (int c = 0; c < C::kColsPerEpiWarp; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(t_acc + c, v);
+        tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            __half2 h = __floats2half2_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
-                                          __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
-            h2[c / 2 + j] = *reinterpret_cast<uint32_t *>(&h);
-          }
+        for (int j = 0; j < 16; ++j) {
+          __half2 h = __floats2half2_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
+                                        __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
+          h2[c / 2 + j] = *reinterpret_cast<uint32_t *>(&h);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty0);
-        if (m < p.M) {
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty0);
+      if (m < p.M) {
 #pragma unroll
-          for (int j = 0; j < C::kColsPerEpiWarp / 8; ++j) {
-            if (n0 + col0 + 8 * j + 8 <= p.N) {
-              uint4 pk;
-              pk.x = h2[4 * j + 0];
-              pk.y = h2[4 * j + 1];
-              pk.z = h2[4 * j + 2];
-              pk.w = h2[4 * j + 3];
-              *reinterpret_cast<uint4 *>(dst + 8 * j) = pk;
-            }
-          }
-        }
-      } else {
-        // 192 columns: each 32-column chunk is stored as soon as it is converted (the
-        // registers do not hold the whole row); the accumulator is released after the last load
-#pragma unroll
-        for (int c = 0; c < C::kColsPerEpiWarp; c += 32) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(t_acc + c, v);
-          tmem_wait_ld();
-          if (c + 32 == C::kColsPerEpiWarp) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty0);
-          }
-          uint32_t h2[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            __half2 h = __floats2half2_rn(__fmul_rn(__uint_as_float(v[2 * j]), alpha),
-                                          __fmul_rn(__uint_as_float(v[2 * j + 1]), alpha));
-            h2[j] = *reinterpret_cast<uint32_t *>(&h);
-          }
-          if (m < p.M) {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              if (n0 + col0 + c + 8 * j + 8 <= p.N) {
-                uint4 pk;
-                pk.x = h2[4 * j + 0];
-                pk.y = h2[4 * j + 1];
-                pk.z = h2[4 * j + 2];
-                pk.w = h2[4 * j + 3];
-                *reinterpret_cast<uint4 *>(dst + c + 8 * j) = pk;
-              }
-            }
+        for (int j = 0; j < C::kColsPerEpiWarp / 8; ++j) {
+          if (n0 + col0 + 8 * j + 8 <= p.N) {
+            uint4 pk;
+            pk.x = h2[4 * j + 0];
+            pk.y = h2[4 * j + 1];
+            pk.z = h2[4 * j + 2];
+            pk.w = h2[4 * j + 3];
+            *reinterpret_cast<uint4 *>(dst + 8 * j) = pk;
           }
         }
       }
