@@ -100,16 +100,11 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
          (static_cast<uint64_t>(2) << 61);
 }
 
-// 4 consecutive TMEM columns of this warp's 32 lanes, all set to v. The store takes a range
-// of four distinct registers, so the value is copied into four temporaries first (naming
-// one register four times leaves columns 1-3 with whatever the neighbouring registers hold).
-__device__ __forceinline__ void tmem_st_x4_rep(uint32_t taddr, uint32_t v) {
-  asm volatile(
-      "{\n\t.reg .b32 t0, t1, t2, t3;\n\t"
-      "mov.b32 t0, %1;\n\tmov.b32 t1, %1;\n\tmov.b32 t2, %1;\n\tmov.b32 t3, %1;\n\t"
-      "tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {t0, t1, t2, t3};\n\t}" ::"r"(taddr),
-      "r"(v)
-      : "memory");
+// One TMEM column of this warp's 32 lanes. The A-operand scale word of lane quarter q is
+// read from column base + q only (the measured layout), so that column is all a scale warp
+// writes for it.
+__device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
 
 // 4 consecutive TMEM columns of this warp's 32 lanes.
@@ -364,7 +359,7 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
         for (int a = 0; a < nk64; ++a) {
           const uint32_t wa =
               *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
-          tmem_st_x4_rep(slot + a * C::kSfaColsPerK64, wa);
+          tmem_st_x1(slot + a * C::kSfaColsPerK64 + q, wa);  // quarter q reads column base + q
           // atom row `lane` holds B rows lane + 32 t' (t' = 0..3) of its 128-row block
           const uint4 b0 = *reinterpret_cast<const uint4 *>(sSfb + a * kSfAtomBytes + lane * 16);
           if constexpr (C::kSfbBlocks == 1) {
@@ -573,9 +568,6 @@ __device__ __forceinline__ bool group_all(bool v, int id, int nthreads) {
 // Named barrier 1: the epilogue warps; 2: the scale warps.
 __device__ __forceinline__ bool epi_all(bool v, int nthreads) { return group_all(v, 1, nthreads); }
 
-__device__ __forceinline__ void tmem_st_x1(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
-}
 
 // The largest E4M3 value <= t, for 0 <= t <= 448 (as an fp32 value). Every E4M3 value is
 // k * 2^E with an integer 0 <= k <= 15, so cutting t to four significant bits (normal range,
@@ -585,8 +577,8 @@ __device__ __forceinline__ float e4m3_floor(float t) {
   return __fmul_rn(floorf(__fmul_rn(t, 512.0f)), 0x1p-9f);
 }
 
-// fp32 activation scales ("Fused Nvfp4 GEMM All Reduce Plugin", input [1]: one fp32 scale
-// per activation block, [B,1,K/16], which the block-scaled MMA cannot take) become NPL planes of
+// fp32 activation scales ("Fused Nvfp4 GEMM All Reduce Plugin": a combined FP32 scale
+// [B,1,K/16] per activation block, which the block-scaled MMA cannot take) become NPL planes of
 // E4M3 codes and one fp32 factor per row: with rho = max_c sa[r,c] / 448 and t = sa * (448 /
 // max) <= 448, plane 1 holds floor_E4M3(t), plane 2 floor_E4M3 of the exact remainder, plane 3
 // the remainder rounded to nearest. Each floor keeps at least four significant bits, so
@@ -887,7 +879,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         for (int a = 0; a < nk64; ++a) {
           const uint32_t wa =
               *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
-          tmem_st_x4_rep(slot + a * 4, wa);
+          tmem_st_x1(slot + a * 4 + q, wa);  // quarter q reads column base + q
           if constexpr (NPL > 1) {
 #pragma unroll
             for (int pl = 0; pl < NPL; ++pl)
@@ -1052,70 +1044,51 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
 //   acc_empty    even CTA; the epilogue warps of both CTAs drained the accumulator (count 16)
 // Every wait is bounded; a cluster barrier opens and closes the kernel so no CTA touches its
 // peer's shared memory before the peer initialised it or after the peer exited.
-template <int STAGES, int BN = 256>
+template <int STAGES>
 struct PairCfg {
-  static constexpr int kN = BN;                         // tile columns
-  static constexpr int kHalf = 128;                     // rows of A per CTA
-  static constexpr int kBRows = BN / 2;                 // rows of B per CTA
+  static constexpr int kN = 256;                        // MMA N (tile columns)
+  static constexpr int kHalf = 128;                     // rows of A and of B per CTA
   static constexpr int kABytes = kHalf * kBKBytes;      // 16 KB
-  static constexpr int kBBytes = kBRows * kBKBytes;     // 16 KB (N = 256) or 24 KB (N = 384)
-  static constexpr int kSfbBlocks = BN / 128;           // B scale atoms: all tile rows
-  static constexpr int kSfaBytes = kK64PerStage * kSfAtomBytes;              // 2 KB
-  static constexpr int kSfbBytes = kSfbBlocks * kK64PerStage * kSfAtomBytes;  // 4 or 6 KB
+  static constexpr int kBBytes = kHalf * kBKBytes;      // 16 KB
+  static constexpr int kSfaBytes = kK64PerStage * kSfAtomBytes;      // 2 KB
+  static constexpr int kSfbBytes = 2 * kK64PerStage * kSfAtomBytes;  // 4 KB (all 256 rows)
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
   static constexpr int kOffSfa = kOffB + STAGES * kBBytes;
   static constexpr int kOffSfb = kOffSfa + STAGES * kSfaBytes;
   static constexpr int kOffBar = kOffSfb + STAGES * kSfbBytes;
-  // tensor-memory scale slots: one per ring stage for N = 256; for N = 384 the accumulator
-  // leaves room for two, reused in turn (sf_empty tells the scale warps a slot was read)
-  static constexpr int kSlots = BN > 256 ? 2 : STAGES;
-  // full[S], sf_ready[S], empty[S], sf_full[slots], sf_empty[slots], acc_full, acc_empty,
-  // tmem slot
-  static constexpr int kBarBytes = (3 * STAGES + 2 * kSlots + 2) * 8 + 16;
+  // full[S], sf_ready[S], sf_full[S], empty[S], acc_full, acc_empty, tmem slot
+  static constexpr int kBarBytes = (4 * STAGES + 2) * 8 + 16;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
-  static constexpr int kAccCols = BN;
-  // a slot: A scales 4 columns per K64 step; B scales of the N = 256 MMA 8 columns per step
-  // (8-aligned bases); for N = 384, those of the N = 128 MMA (tile columns 256..383) 4 more
+  static constexpr int kAccCols = kN;
   static constexpr int kSfaColsPerK64 = 4;
-  static constexpr int kSfb1ColsPerK64 = 8;
-  static constexpr int kSfb2ColsPerK64 = BN > 256 ? 4 : 0;
-  static constexpr int kSlotB1 = kK64PerStage * kSfaColsPerK64;
-  static constexpr int kSlotB2 = kSlotB1 + kK64PerStage * kSfb1ColsPerK64;
-  static constexpr int kSlotCols = kSlotB2 + kK64PerStage * kSfb2ColsPerK64;
+  static constexpr int kSfbColsPerK64 = 8;
+  static constexpr int kSlotCols = kK64PerStage * (kSfaColsPerK64 + kSfbColsPerK64);
   static constexpr int kSfCol0 = kAccCols;
   static constexpr int kTmemCols = 512;
-  // epilogue: three warps per lane quarter for N = 384, two for 256: 128 columns each, so
-  // every warp holds its whole share in registers before it releases the accumulator
-  static constexpr int kEpiWarps = BN / 32;
+  static constexpr int kEpiWarps = 8;
   static constexpr int kColsPerEpiWarp = kN * 4 / kEpiWarps;  // 128
   static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
-  static_assert(BN == 256 || BN == 384, "pair tile width");
-  static_assert(kSfCol0 + kSlots * kSlotCols <= kTmemCols, "TMEM columns");
+  static_assert(kSfCol0 + STAGES * kSlotCols <= kTmemCols, "TMEM columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
   // kind::mxf4nvf4: E2M1 A and B, K-major, UE4M3 scales; N >> 3 at bit 17, M >> 4 at bit 24
-  static constexpr uint32_t idesc(int n) {
-    return (1u << 7) | (1u << 10) | (uint32_t(n >> 3) << 17) | (uint32_t(256 >> 4) << 24);
-  }
-  static constexpr uint32_t kIdesc = idesc(256);
-  static constexpr uint32_t kIdesc2 = idesc(128);
+  static constexpr uint32_t kIdesc =
+      (1u << 7) | (1u << 10) | (uint32_t(kN >> 3) << 17) | (uint32_t(256 >> 4) << 24);
 };
 
-template <int STAGES, int BN>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>::kThreads, 1)
+template <int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kThreads, 1)
     gemm_nvfp4_pair_kernel(const __grid_constant__ CUtensorMap tmap_a,
                            const __grid_constant__ CUtensorMap tmap_b, const KernelParams p) {
-  using C = PairCfg<STAGES, BN>;
-  constexpr bool kRing = C::kSlots != STAGES;  // scale slots reused independently of stages
+  using C = PairCfg<STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *sf_ready = full + STAGES;
-  uint64_t *empty = sf_ready + STAGES;
-  uint64_t *sf_full = empty + STAGES;
-  uint64_t *sf_empty = sf_full + C::kSlots;
-  uint64_t *acc_full = sf_empty + C::kSlots;
+  uint64_t *sf_full = sf_ready + STAGES;
+  uint64_t *empty = sf_full + STAGES;
+  uint64_t *acc_full = empty + STAGES;
   uint64_t *acc_empty = acc_full + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
 
@@ -1135,11 +1108,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 2);
       mbar_init(&sf_ready[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&sf_full[s], 8);
-      mbar_init(&sf_empty[s], 1);
+      mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * C::kEpiWarps);
@@ -1169,9 +1139,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
     for (int t = pair; t < num_tiles && ok; t += npairs) {
       int64_t m0, n0;
       tile_origin(t, m0, n0);
-      const int64_t arow = m0 + C::kHalf * rank;  // this CTA's A rows
+      const int64_t arow = m0 + C::kHalf * rank;  // this CTA's A rows and B rows
+      const int64_t brow = n0 + C::kHalf * rank;
       int sfb_copies = 0;
-      for (int blk = 0; blk < C::kSfbBlocks; ++blk)
+      for (int blk = 0; blk < 2; ++blk)
         if ((n0 / 128 + blk) * 128 < p.sfb_rows_padded) ++sfb_copies;
       const bool sfa_copy = arow < p.sfa_rows_padded;
       for (int kt = 0; kt < num_kt; ++kt, ++it) {
@@ -1205,19 +1176,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
           const uint32_t fullc = full0 + stage * 8;
           mbar_arrive_expect_tx_cluster(fullc, C::kABytes + C::kBBytes);
           tma_load_2d_pair(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(arow), fullc);
-          if constexpr (BN == 256) {
-            // B rows [128 r, 128 r + 128) of the tile
-            tma_load_2d_pair(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(n0 + 128 * rank), fullc);
-          } else {
-            // rows [128 r, 128 r + 128) for the N = 256 MMA, then [256 + 64 r, 256 + 64 r + 64)
-            // for the N = 128 MMA, in 64-row boxes
-            const int64_t b1 = n0 + 128 * rank;
-            tma_load_2d_pair(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(b1), fullc);
-            tma_load_2d_pair(sB + 64 * kBKBytes, &tmap_b, kt * kBKBytes, static_cast<int32_t>(b1 + 64),
-                             fullc);
-            tma_load_2d_pair(sB + 128 * kBKBytes, &tmap_b, kt * kBKBytes,
-                             static_cast<int32_t>(n0 + 256 + 64 * rank), fullc);
-          }
+          tma_load_2d_pair(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(brow), fullc);
         }
         __syncwarp();
       }
@@ -1244,41 +1203,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
           break;
         }
         tc_fence_after();
-        int64_t prev = -1;  // iteration whose releases are still to be issued (one stage late)
+        int prev = -1;  // stage whose release is still to be issued (see the single-CTA kernel)
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int stage = static_cast<int>(it % STAGES);
           const uint32_t round = it / STAGES;
-          const int slot = static_cast<int>(it % C::kSlots);
           if (!mbar_wait_cluster(&full[stage], round & 1, kWaitTimeoutNs) ||
-              !mbar_wait_cluster(&sf_full[slot], (it / C::kSlots) & 1, kWaitTimeoutNs)) {
+              !mbar_wait_cluster(&sf_full[stage], round & 1, kWaitTimeoutNs)) {
             report_timeout(p.dev_status);
             ok = false;
             break;
           }
           tc_fence_after();
-          if (prev >= 0) {
-            tc_commit_pair(&empty[prev % STAGES], 0x3);
-            if constexpr (kRing) tc_commit_pair(&sf_empty[prev % C::kSlots], 0x3);
-          }
+          if (prev >= 0) tc_commit_pair(&empty[prev], 0x3);
           const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
           const uint32_t sA = smem_u32(smem + C::kOffA + stage * C::kABytes);
           const uint32_t sB = smem_u32(smem + C::kOffB + stage * C::kBBytes);
-          const uint32_t sc = tmem_base + C::kSfCol0 + slot * C::kSlotCols;
+          const uint32_t slot = tmem_base + C::kSfCol0 + stage * C::kSlotCols;
           for (int a = 0; a < nk64; ++a) {
-            const uint32_t acc = (kt | a) != 0 ? 1u : 0u;
             mma_nvf4_pair(tmem_base, desc_sw128(sA + a * 32), desc_sw128(sB + a * 32), C::kIdesc,
-                          sc + a * C::kSfaColsPerK64, sc + C::kSlotB1 + a * C::kSfb1ColsPerK64, acc);
-            if constexpr (BN > 256)
-              mma_nvf4_pair(tmem_base + 256, desc_sw128(sA + a * 32),
-                            desc_sw128(sB + 128 * kBKBytes + a * 32), C::kIdesc2,
-                            sc + a * C::kSfaColsPerK64, sc + C::kSlotB2 + a * C::kSfb2ColsPerK64, acc);
+                          slot + a * C::kSfaColsPerK64,
+                          slot + kK64PerStage * C::kSfaColsPerK64 + a * C::kSfbColsPerK64,
+                          (kt | a) != 0 ? 1u : 0u);
           }
-          prev = it;
+          prev = stage;
         }
-        if (prev >= 0) {
-          tc_commit_pair(&empty[prev % STAGES], 0x3);
-          if constexpr (kRing) tc_commit_pair(&sf_empty[prev % C::kSlots], 0x3);
-        }
+        if (prev >= 0) tc_commit_pair(&empty[prev], 0x3);
         if (ok) tc_commit_pair(acc_full, 0x3);
       }
     }
@@ -1294,46 +1243,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
       for (int kt = 0; kt < num_kt; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
-        const int slot = static_cast<int>(it % C::kSlots);
         if (!mbar_wait_warp(&sf_ready[stage], round & 1, kWaitTimeoutNs)) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
           break;
         }
-        if constexpr (kRing) {
-          // the MMAs that read this slot two iterations ago have completed
-          if (it >= static_cast<uint32_t>(C::kSlots) &&
-              !mbar_wait_warp(&sf_empty[slot], (it / C::kSlots - 1) & 1, kWaitTimeoutNs)) {
-            if (lane == 0) report_timeout(p.dev_status);
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
         const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
         const uint8_t *sSfa = smem + C::kOffSfa + stage * C::kSfaBytes;
         const uint8_t *sSfb = smem + C::kOffSfb + stage * C::kSfbBytes;
-        const uint32_t sc = lane_base + C::kSfCol0 + slot * C::kSlotCols;
-        // same tensor-memory scale layout as the single-CTA kernel with a 256-row B operand;
-        // the N = 128 MMA's B rows (the third atom block) take 4 columns of their own
+        const uint32_t slot = lane_base + C::kSfCol0 + stage * C::kSlotCols;
+        const uint32_t slot_b = slot + kK64PerStage * C::kSfaColsPerK64;
+        // same tensor-memory scale layout as the single-CTA kernel with a 256-row B operand
         for (int a = 0; a < nk64; ++a) {
           const uint32_t wa =
               *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
-          tmem_st_x4_rep(sc + a * C::kSfaColsPerK64, wa);
+          tmem_st_x1(slot + a * C::kSfaColsPerK64 + q, wa);  // quarter q reads column base + q
           const uint4 b0 = *reinterpret_cast<const uint4 *>(sSfb + a * kSfAtomBytes + lane * 16);
           const uint4 b1 = *reinterpret_cast<const uint4 *>(
               sSfb + (kK64PerStage + a) * kSfAtomBytes + lane * 16);
-          tmem_st_x8(sc + C::kSlotB1 + a * C::kSfb1ColsPerK64, b0, b1);
-          if constexpr (BN > 256) {
-            const uint4 b2 = *reinterpret_cast<const uint4 *>(
-                sSfb + (2 * kK64PerStage + a) * kSfAtomBytes + lane * 16);
-            tmem_st_x4(sc + C::kSlotB2 + a * C::kSfb2ColsPerK64, b2.x, b2.y, b2.z, b2.w);
-          }
+          tmem_st_x8(slot_b + a * C::kSfbColsPerK64, b0, b1);
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(sf_full0 + slot * 8);
+        if (lane == 0) mbar_arrive_cluster(sf_full0 + stage * 8);
       }
     }
   } else if (warp >= kEpiWarp0) {
@@ -1354,9 +1287,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
       }
       tc_fence_after();
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col0;
-      const int64_t m = m0 + C::kHalf * rank + row;
-      __half *dst = p.out + m * p.N + n0 + col0;
-      // all 128 columns into registers, release the accumulator, then store
       uint32_t h2[C::kColsPerEpiWarp / 2];
 #pragma unroll
       for (int c = 0; c < C::kColsPerEpiWarp; c += 32) {
@@ -1373,7 +1303,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES, BN>:
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty0);
+      const int64_t m = m0 + C::kHalf * rank + row;
       if (m < p.M) {
+        __half *dst = p.out + m * p.N + n0 + col0;
 #pragma unroll
         for (int j = 0; j < C::kColsPerEpiWarp / 8; ++j) {
           if (n0 + col0 + 8 * j + 8 <= p.N) {
@@ -1543,7 +1475,7 @@ static cudaError_t run(const GemmArgs &g, int num_sms, cudaStream_t st) {
 
 // CTA pairs that can be resident at once (a pair needs two SMs of one GPC, so this can be
 // below half the SM count); the persistent grid never exceeds it. Queried once per device.
-template <int STAGES, int BN>
+template <int STAGES>
 static int resident_pairs() {
   constexpr int kMaxDevices = 64;
   static std::once_flag once[kMaxDevices];
@@ -1551,9 +1483,9 @@ static int resident_pairs() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
   std::call_once(once[dev], [dev]() {
-    using C = PairCfg<STAGES, BN>;
+    using C = PairCfg<STAGES>;
     pairs[dev] = 0;
-    if (ensure_smem_attr(gemm_nvfp4_pair_kernel<STAGES, BN>, C::kSmemBytes) != cudaSuccess) return;
+    if (ensure_smem_attr(gemm_nvfp4_pair_kernel<STAGES>, C::kSmemBytes) != cudaSuccess) return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(C::kThreads, 1, 1);
@@ -1566,20 +1498,21 @@ static int resident_pairs() {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<STAGES, BN>, &cfg) == cudaSuccess)
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_pair_kernel<STAGES>, &cfg) == cudaSuccess)
       pairs[dev] = n;
   });
   return pairs[dev];
 }
 
-template <int STAGES, int BN>
-static cudaError_t run_pair(const GemmArgs &g, cudaStream_t st) {
-  using C = PairCfg<STAGES, BN>;
+template <int STAGES>
+static cudaError_t run_pair(const GemmArgs &g, int num_sms, cudaStream_t st) {
+  (void)num_sms;
+  using C = PairCfg<STAGES>;
   CUtensorMap ma, mb;
   KernelParams p{};
   const int64_t kb = g.K / 2;
   if (!make_operand_map(&ma, g.a_q, g.M, kb, C::kHalf)) return cudaErrorInvalidValue;
-  if (!make_operand_map(&mb, g.w_q, g.N, kb, BN == 256 ? 128 : 64)) return cudaErrorInvalidValue;
+  if (!make_operand_map(&mb, g.w_q, g.N, kb, C::kHalf)) return cudaErrorInvalidValue;
   p.sfa = g.a_sf;
   p.sfb = g.w_sf;
   p.sfb_8x4 = 0;
@@ -1596,26 +1529,12 @@ static cudaError_t run_pair(const GemmArgs &g, cudaStream_t st) {
   p.tiles_a = static_cast<int>((g.M + 255) / 256);
   p.tiles_b = static_cast<int>((g.N + C::kN - 1) / C::kN);
   const int64_t tiles = static_cast<int64_t>(p.tiles_a) * p.tiles_b;
-  const int resident = resident_pairs<STAGES, BN>();
+  const int resident = resident_pairs<STAGES>();
   if (resident <= 0) return cudaErrorLaunchOutOfResources;
   const int64_t pairs = tiles < resident ? tiles : resident;
-  gemm_nvfp4_pair_kernel<STAGES, BN>
-      <<<static_cast<int>(2 * pairs), C::kThreads, C::kSmemBytes, st>>>(ma, mb, p);
+  gemm_nvfp4_pair_kernel<STAGES><<<static_cast<int>(2 * pairs), C::kThreads, C::kSmemBytes, st>>>(
+      ma, mb, p);
   return cudaGetLastError();
-}
-
-// Pair tile width by the operand bytes a CTA pair stages per wave: a 256 x BN tile stages
-// (256 + BN) rows of K, and the tiles run in waves over the resident pairs, so the bytes go as
-// waves x (256 + BN). The 384 tile's 13% byte saving mostly does not show up as time: on B200
-// it measured 2% faster at 8192^3 and 1% slower at 4096 x 4096 x 8192, with the scale-slot
-// ring ruled out as the cause. It is taken only where the model gives it 10% or more.
-static int pair_tile_width(int64_t M, int64_t N, int resident256, int resident384) {
-  if (resident256 <= 0 || resident384 <= 0) return 256;
-  const int64_t ta = (M + 255) / 256;
-  const int64_t t256 = ta * ((N + 255) / 256), t384 = ta * ((N + 383) / 384);
-  const int64_t c256 = (t256 + resident256 - 1) / resident256 * (256 + 256);
-  const int64_t c384 = (t384 + resident384 - 1) / resident384 * (256 + 384);
-  return c384 * 10 <= c256 * 9 ? 384 : 256;
 }
 
 // Small-M stream-K layout for a device with num_sms SMs: grid, pieces per tile, workspace.
@@ -1720,9 +1639,7 @@ cudaError_t launch_gemm(const GemmArgs &g, int num_sms, cudaStream_t st) {
     return run<32, 6, true>(g, num_sms, st);
   }
   if (g.M < 256 || num_sms < 2) return run<256, 4, false>(g, num_sms, st);
-  if (pair_tile_width(g.M, g.N, resident_pairs<5, 256>(), resident_pairs<4, 384>()) == 384)
-    return run_pair<4, 384>(g, st);
-  return run_pair<5, 256>(g, st);
+  return run_pair<5>(g, num_sms, st);
 }
 
 }  // namespace nvfp4

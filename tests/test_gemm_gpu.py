@@ -52,10 +52,9 @@ def _run(nv, ops, a_layout):
     return out.cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-# M <= 32: swap-AB tiles; 33..255: single-CTA 128 x 256 tiles; M >= 256: CTA-pair tiles,
-# 256 x 256, or 256 x 384 where that needs fewer operand bytes per wave (4096 x 2560,
-# 2000 x 5000, 1536 x 4608, 2048 x 3072 on 148 SMs); ragged M, N and K tails, and more tiles
-# than resident pairs so the accumulator and the scale slots are reused.
+# M <= 32: swap-AB tiles; 33..255: single-CTA 128 x 256 tiles; M >= 256: CTA-pair 256 x 256
+# tiles (ragged M, N and K tails, and more tiles than resident pairs so the accumulator is
+# reused).
 SMALL = [(1, 256, 512), (8, 256, 512), (16, 256, 512), (32, 512, 1024), (3, 136, 64),
          (33, 256, 512), (128, 256, 256), (130, 520, 320), (256, 1024, 2048), (300, 264, 4096),
          (520, 776, 320), (4096, 2560, 512), (2000, 5000, 320), (1536, 4608, 512),
@@ -316,7 +315,7 @@ def test_gemm_bit_exact_when_accumulation_is_exact(M, N, K):
     1/16 below 2^8, so every partial sum of K = 512 terms is exact in fp32 whatever the
     accumulation order, and alpha = 1: the kernels' fp16 output must equal the oracle's single
     rounding of the exact sum bit for bit. Shapes reach the decode (split-K), single-CTA and
-    both CTA-pair kernels."""
+    CTA-pair kernels."""
     nv = require_cuda()
     rng = np.random.default_rng(M + N)
     a = workloads.random_bytes((M, K // 2), M + 1)
