@@ -14,17 +14,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
-// One lane of the warp returns true (the lowest active one).
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred = 0;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t"
-      "elect.sync _|P, 0xffffffff;\n\t"
-      "selp.b32 %0, 1, 0, P;\n\t}"
-      : "=r"(pred));
-  return pred != 0;
-}
-
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -40,10 +29,6 @@ __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
 // Makes barrier initialisation visible to the async proxy (TMA, tcgen05).
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
@@ -81,31 +66,6 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   }
 }
 
-// try_wait with an explicit suspend-time hint: a thread whose phase is not complete sleeps
-// until the phase completes or about `hint_ns` pass, instead of retrying after the short
-// system-dependent default; waiting warps then take no issue slots from working ones.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
-      "selp.b32 %0, 1, 0, P;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait built on the sleeping try_wait; gives up (returns false) after timeout_ns.
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
-                                                uint32_t hint_ns) {
-  if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
-    if (globaltimer_ns() - t0 > timeout_ns) return false;
-  }
-}
 
 // Whole-warp form of mbar_wait_bounded: every lane waits, then the warp reconverges and
 // agrees on the outcome, so warp-collective (.sync.aligned) instructions that follow run
@@ -179,13 +139,6 @@ __device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint6
       "p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
-}
-
-// Copies a 32-row x 128-bit shared-memory matrix into TMEM, replicated into all four
-// 32-lane sub-partitions.
-__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t src_desc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc)
-               : "memory");
 }
 
 // Arrives on `bar` once every tcgen05 operation issued so far by this thread completes.
@@ -340,17 +293,6 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
 
 // ------------------------------------------------------------------------------ FP4 / FP8
 
-// Two fp32 -> one byte of two E2M1 codes (round to nearest even, saturate):
-// `lo` goes to bits 3:0, `hi` to bits 7:4.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint32_t out;
-  asm("{\n\t.reg .b8 t;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-      "cvt.u32.u8 %0, t;\n\t}"
-      : "=r"(out)
-      : "f"(hi), "f"(lo));
-  return out;
-}
 
 // fp32 -> E4M3 code (round to nearest even, saturate to +-448).
 __device__ __forceinline__ uint32_t cvt_e4m3(float v) {

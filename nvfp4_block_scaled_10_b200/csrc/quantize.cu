@@ -54,25 +54,6 @@ __device__ __forceinline__ int64_t sf_offset(int layout, int64_t r, int64_t c, i
   return r * C + c;
 }
 
-// Quantizes 16 fp32 values with encode scale g. Returns the 8 packed bytes (element 2j in
-// the low nibble of byte j) and the E4M3 scale code.
-__device__ __forceinline__ uint64_t quant_block16(const float (&y)[16], float g, uint32_t &s_enc) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(y[i]));
-  const float s = __fmul_rn(__fdiv_rn(amax, 6.0f), g);
-  s_enc = cvt_e4m3(s);
-  const float s_dec = e4m3_to_f32(s_enc);
-  const float r = (s_dec == 0.0f) ? 0.0f : fminf(__fdiv_rn(g, s_dec), FLT_MAX);
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    lo |= cvt_e2m1x2(__fmul_rn(y[2 * j], r), __fmul_rn(y[2 * j + 1], r)) << (8 * j);
-    hi |= cvt_e2m1x2(__fmul_rn(y[8 + 2 * j], r), __fmul_rn(y[8 + 2 * j + 1], r)) << (8 * j);
-  }
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
 // fl(x / 6) for x >= 0 (a block maximum), the IEEE quotient, without the general division
 // sequence: q0 = fl(x * fl(1/6)), rem = x - 6*q0 by one FMA, q1 = q0 + rem*fl(1/6) by one
 // FMA. An exhaustive check over every fp32 bit pattern with a clear sign bit finds q1
