@@ -133,3 +133,16 @@ def test_gemm_act_f32_argument_checks(L):
     assert g(P16, P16, P16, P16, ctypes.c_void_p(0x10002), P16, 16, 256, 512, None, 0, None,
              None) == nv.ERR_MISALIGNED                                        # w_scale
     assert g(*a, 0, 256, 512, None, 0, None, None) == nv.OK                    # empty
+
+
+def test_missing_library_fails_loudly(monkeypatch):
+    """No fallback: without the built library every entry point raises, on a GPU machine too."""
+    import torch
+
+    monkeypatch.setattr(nv, "LIB_PATH", os.path.join(ROOT, "no_such_dir", "libnvfp4.so"))
+    monkeypatch.setattr(nv, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        nv.lib()
+    x = torch.zeros(4, 32, dtype=torch.bfloat16)
+    with pytest.raises(RuntimeError, match="not built"):
+        nv.nvfp4_quantize(x, torch.ones(1))
