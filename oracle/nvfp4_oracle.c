@@ -32,10 +32,11 @@
  *    weight scale, FP16 [B,N] result): "Fused Nvfp4 GEMM All Reduce Plugin"
  *    (TensorRT-Edge-LLM C++ API), input/output tensor list.
  *
- * Parity pins live in tests/test_oracle_*.py. Function without an external pin:
- *  - the 8x4 byte order (orc_sf_offset, layout 2) is a reading; it is checked only against a
- *    second formulation of the same reading (reshape/transpose) and for bijection:
- *    "parity unpinned" for the 8x4 byte order itself.
+ * Parity pins live in tests/test_oracle_*.py. The 8x4 byte order (orc_sf_offset, layout 2)
+ * is a reading, since the pages name the layout without its bytes. On CPU it is checked
+ * against a second formulation of the same reading and for bijection; on the GPU both
+ * swizzled layouts are checked against FlashInfer's fp4_quantize, the library of "feature:
+ * add fp4 mm using trtllm backend" (tests/test_layout_library_gpu.py).
  */
 #include <float.h>
 #include <math.h>
