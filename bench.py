@@ -307,7 +307,7 @@ def run_ours(args, rank, world, torch, dist):
             ws_bytes = nv.nvfp4_gemm_act_f32_workspace_bytes(M, N, K)
         else:
             ws_bytes = nv.nvfp4_gemm_workspace_bytes(M, N, K)
-        gemm_ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+        gemm_ws = torch.zeros(max(ws_bytes, 16), dtype=torch.uint8, device=dev)  # zero on first use
 
         def gemm_call(aq, asf, wq, wsf, ws):
             if wl == "decode_f32":

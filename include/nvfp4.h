@@ -195,11 +195,14 @@ NVFP4_API int nvfp4_sf_unswizzle(const uint8_t *in, uint8_t *lin, int64_t R, int
 /*
  * Workspace bytes nvfp4_gemm needs for this shape on the current device. Non-zero only for
  * M <= 32 (K <= 24576): that path splits the K range of the weight tiles evenly over the
- * SMs ("stream-K") and keeps fp32 partial tiles [tiles][pieces][128][32] plus one int
- * arrival counter per 128-row weight tile there (about 7.4 MB for N = 28672, K = 8192 on
- * 148 SMs). The contents need no initialisation and are scratch after the call; calls that
- * share a workspace must not overlap on the GPU. Returns 0 when no device is current.
- * Host only.
+ * SMs ("stream-K") and keeps one int arrival counter per 128-row weight tile (at the front,
+ * in 16 * (workspace_bytes / 65536 + 1) bytes whatever the shape) and fp32 partial tiles
+ * [tiles][pieces][128][32] after them (about 7.4 MB for N = 28672, K = 8192 on 148 SMs).
+ * Pass the same workspace_bytes with a given buffer. The workspace must be zero-filled
+ * before its first use (cudaMemset once); every
+ * call that completes leaves the counters zero again, so it needs no per-call reset. After
+ * a call reports an error in dev_status, zero it again. Calls that share a workspace must
+ * not overlap on the GPU. Returns 0 when no device is current. Host only.
  */
 NVFP4_API size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
@@ -218,12 +221,13 @@ NVFP4_API size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * w_q      device, [N, K/2] packed E2M1.   w_sf device, 128x4 layout.   w_g device fp32.
  * out      device, [M, N] fp16, row-major, row stride N.
  * workspace/workspace_bytes: device, 16-byte aligned, >= nvfp4_gemm_workspace_bytes(M, N,
- *          K) (NVFP4_ERR_INVALID_ARG when smaller); may be NULL when that is 0. The call
- *          resets the counters it uses with an asynchronous memset on `stream` before the
- *          kernel.
+ *          K) (NVFP4_ERR_INVALID_ARG when smaller); may be NULL when that is 0. Zero-filled
+ *          before its first use; each completed call leaves it zero-filled (see
+ *          nvfp4_gemm_workspace_bytes).
  * dev_status: device int32 or NULL. Each bounded wait inside the kernel that gives up
  *          (about 2 s without progress) ORs 1 into it and the kernel returns without
- *          finishing; the caller reads it after synchronizing (NVFP4_ERR_TIMEOUT).
+ *          finishing; a split-K tile counter found non-zero on entry (a workspace that was
+ *          not zero-filled) ORs 4. The caller reads it after synchronizing.
  * Requires: K % 64 == 0, N % 8 == 0, a_q/w_q/a_sf/w_sf/out 16-byte aligned, a_layout in
  *          {128x4, 8x4} (8x4 only when M <= 32).
  */
@@ -270,7 +274,8 @@ NVFP4_API int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int 
  * workspace/workspace_bytes: device, 16-byte aligned, >= nvfp4_gemm_act_f32_workspace_bytes
  *          (M, N, K); same use as in nvfp4_gemm.
  * dev_status: device int32 or NULL; bit 1 a bounded wait gave up (NVFP4_ERR_TIMEOUT), bit 2
- *          a bad activation scale. The caller reads it after synchronizing.
+ *          a bad activation scale, bit 4 a workspace that was not zero-filled. The caller
+ *          reads it after synchronizing.
  * Requires: K % 64 == 0, N % 8 == 0.
  */
 NVFP4_API size_t nvfp4_gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K);

@@ -233,7 +233,7 @@ def nvfp4_gemm(a_q: torch.Tensor, a_sf: torch.Tensor, a_g: torch.Tensor, w_q: to
         out = torch.empty(M, N, dtype=torch.float16, device=a_q.device)
     nbytes = nvfp4_gemm_workspace_bytes(M, N, K)
     if workspace is None and nbytes > 0:
-        workspace = torch.empty(nbytes, dtype=torch.uint8, device=a_q.device)
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=a_q.device)  # zero on first use
     if per_token_a and a_g.numel() != M:
         raise ValueError(f"per_token_a needs a_g with M = {M} elements, got {a_g.numel()}")
     fn = lib().nvfp4_gemm_per_token if per_token_a else lib().nvfp4_gemm
@@ -263,7 +263,7 @@ def nvfp4_gemm_act_f32(a_q: torch.Tensor, a_sf32: torch.Tensor, w_q: torch.Tenso
         out = torch.empty(M, N, dtype=torch.float16, device=a_q.device)
     nbytes = nvfp4_gemm_act_f32_workspace_bytes(M, N, K)
     if workspace is None and nbytes > 0:
-        workspace = torch.empty(nbytes, dtype=torch.uint8, device=a_q.device)
+        workspace = torch.zeros(nbytes, dtype=torch.uint8, device=a_q.device)  # zero on first use
     _check(lib().nvfp4_gemm_act_f32(_ptr(a_q), _ptr(a_sf32), _ptr(w_q), _ptr(w_sf), _ptr(w_scale),
                                     _ptr(out), M, N, K, _ptr(workspace),
                                     0 if workspace is None else workspace.numel(),

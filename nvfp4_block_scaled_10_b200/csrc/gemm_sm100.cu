@@ -474,7 +474,8 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
 // per CTA, so every CTA streams the same amount of weight bytes whatever the tile count.
 // A CTA whose range covers only part of a tile's K writes its fp32 partial accumulator to
 // the workspace; the last CTA to finish a tile (a per-tile arrival counter) adds the pieces
-// in piece order (deterministic) and writes the fp16 result. Activation scales: with the
+// in piece order (deterministic), writes the fp16 result and zeroes the counter again, so a
+// workspace zero-filled once stays ready for the next call with no memset node per call. Activation scales: with the
 // 8x4 layout the <= 32 rows of all K (K/16 bytes each, four contiguous 8-row blocks) are
 // copied into shared memory once per CTA; with the 128x4 layout the activation atoms of
 // each ring stage are copied with the weight atoms.
@@ -533,7 +534,7 @@ struct DecParams {
   int tiles;            // 128-row weight tiles
   int max_pieces;       // CTAs a tile's K range can be split over
   float *partials;      // [tiles][max_pieces][128][32] fp32
-  int *counters;        // [tiles], zero on entry
+  int *counters;        // [tiles], zero on entry and zeroed again by each tile's last arriver
   int32_t *dev_status;
   const float *a_sf32;  // NPL = 3: fp32 activation scales [M, K/16]
   const float *w_scale; // NPL = 3: fp32 weight dequantization scale (multiplies)
@@ -980,6 +981,10 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         __threadfence();
         const int old = atomicAdd(p.counters + tile, 1);
         *last_flag = (old == pieces - 1) ? 1 : 0;
+        // the last arriver hands the counter back zeroed for the next call on this
+        // workspace; a count past the pieces means the workspace was not zero on entry
+        if (old == pieces - 1) atomicExch(p.counters + tile, 0);
+        if ((old < 0 || old >= pieces) && p.dev_status != nullptr) atomicOr(p.dev_status, kDevErrWorkspace);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(C::kEpiWarps * 32) : "memory");
       const bool last = *last_flag != 0;
@@ -1543,9 +1548,22 @@ struct DecPlan {
   int tiles = 0;
   int max_pieces = 0;
   size_t partial_bytes = 0;
-  size_t counter_bytes = 0;
   bool usable = false;
 };
+
+// Workspace layout: the tile counters first, in a region sized by the workspace length alone,
+// then the fp32 partial tiles. Every partial tile takes 16 KB, so a workspace of W bytes
+// serves at most W / 16384 tiles and 16 * (W / 65536 + 1) bytes hold all their counters:
+// whatever shape uses the workspace, its counters fall in this region and no call's partial
+// tiles ever overwrite another shape's counters. The last arriver of every split tile
+// zeroes its counter, so a workspace zero-filled once stays valid call after call.
+static size_t counter_region(size_t W) { return 16 * (W / 65536 + 1); }
+
+// Smallest workspace whose space after the counter region holds P bytes of partials; any
+// larger one does too (counter_region(W) <= W / 4096 + 16).
+static size_t workspace_for(size_t P) {
+  return P == 0 ? 0 : (P + 16) + (P + 16 + 4094) / 4095 + 16;
+}
 
 static DecPlan dec_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool sfb_fits = true) {
   DecPlan d;
@@ -1560,7 +1578,6 @@ static DecPlan dec_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool sfb_f
   if (mp > num_kt) mp = num_kt;
   d.max_pieces = static_cast<int>(mp);
   d.partial_bytes = static_cast<size_t>(d.tiles) * d.max_pieces * kBM * kDecBN * sizeof(float);
-  d.counter_bytes = (static_cast<size_t>(d.tiles) * sizeof(int) + 255) / 256 * 256;
   d.usable = true;
   return d;
 }
@@ -1569,12 +1586,12 @@ static bool sfb_8x4_fits(int64_t K) { return K / 64 * 128 <= kDecMaxSfbBytes; }
 
 size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   const DecPlan d = dec_plan(M, N, K, num_sms, sfb_8x4_fits(K));
-  return d.usable ? d.partial_bytes + d.counter_bytes : 0;
+  return d.usable ? workspace_for(d.partial_bytes) : 0;
 }
 
 size_t gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   const DecPlan d = dec_plan(M < kDecBN ? M : kDecBN, N, K, num_sms);
-  return d.usable ? d.partial_bytes + d.counter_bytes : 0;
+  return d.usable ? workspace_for(d.partial_bytes) : 0;
 }
 
 template <int STAGES, int NPL = 1>
@@ -1600,11 +1617,11 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   p.K = g.K;
   p.tiles = d.tiles;
   p.max_pieces = d.max_pieces;
-  p.partials = static_cast<float *>(g.workspace);
-  p.counters = reinterpret_cast<int *>(static_cast<uint8_t *>(g.workspace) + d.partial_bytes);
+  p.counters = static_cast<int *>(g.workspace);
+  p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(g.workspace) +
+                                         counter_region(g.workspace_bytes));
   p.dev_status = g.dev_status;
-  cudaError_t e = cudaMemsetAsync(p.counters, 0, d.counter_bytes, st);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
   const int smem = C::smem_bytes(static_cast<int>(g.K / 64), p.a_sf_8x4 != 0);
   e = ensure_smem_attr(gemm_nvfp4_decode_kernel<STAGES, NPL>, smem);
   if (e != cudaSuccess) return e;

@@ -16,6 +16,7 @@ constexpr int kInFp16 = 1;
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s without progress
 constexpr int kDevErrTimeout = 1;
 constexpr int kDevErrBadScale = 2;  // an fp32 activation scale was negative, NaN or infinite
+constexpr int kDevErrWorkspace = 4;  // a split-K tile counter was not zero when the call began
 
 // quantize.cu
 int *device_error_symbol();

@@ -382,3 +382,49 @@ def test_row_parallel_nccl_one_rank():
         assert torch.equal(got, ref)
     finally:
         dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ split-K workspace reuse
+
+def test_workspace_reused_across_calls_stays_zero():
+    """One zero-filled workspace serves consecutive small-M calls of different shapes (each
+    against the oracle); the tiles' last arrivers hand it back zero-filled every time."""
+    nv = require_cuda()
+    ws = torch.zeros(max(nv.nvfp4_gemm_workspace_bytes(32, 20480, 8192),
+                         nv.nvfp4_gemm_act_f32_workspace_bytes(40, 20480, 8192)),
+                     dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for i, (M, N, K) in enumerate([(8, 20480, 1024), (32, 4096, 3072), (1, 20480, 8192),
+                                   (17, 1032, 8192), (32, 4096, 3072)]):
+        ops = _random_operands(M, N, K, seed=600 + i)
+        _, ref = orc.gemm(*ops, want_f64=True)
+        d = _to_device(nv, *ops, orc.L8x4 if i % 2 else orc.L128x4)
+        out = nv.nvfp4_gemm(**d, workspace=ws, dev_status=status)
+        torch.cuda.synchronize()
+        gemm_close(out.cpu().view(torch.int16).numpy().view(np.uint16), ref)
+        assert status.item() == 0
+    # the counters sit at the front, in a region sized by the workspace length alone
+    region = 16 * (ws.numel() // 65536 + 1)
+    assert int(ws[:region].count_nonzero().item()) == 0
+
+
+def test_workspace_not_zero_is_flagged():
+    """A workspace whose tile counters are not zero on entry is reported (dev_status bit 4),
+    and the same workspace zero-filled again gives the right result."""
+    nv = require_cuda()
+    M, N, K = 8, 20480, 1024
+    ops = _random_operands(M, N, K, seed=77)
+    _, ref = orc.gemm(*ops, want_f64=True)
+    d = _to_device(nv, *ops, orc.L128x4)
+    ws = torch.full((nv.nvfp4_gemm_workspace_bytes(M, N, K),), 0x7F, dtype=torch.uint8,
+                    device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvfp4_gemm(**d, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() & 4
+    ws.zero_()
+    status.zero_()
+    out = nv.nvfp4_gemm(**d, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    gemm_close(out.cpu().view(torch.int16).numpy().view(np.uint16), ref)
