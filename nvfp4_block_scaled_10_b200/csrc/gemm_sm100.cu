@@ -532,12 +532,16 @@ struct DecParams {
   __half *out;
   int64_t M, N, K;
   int tiles;            // 128-row weight tiles
-  int max_pieces;       // CTAs a tile's K range can be split over
-  float *partials;      // [tiles][max_pieces][128][32] fp32
+  int max_pieces;       // CTAs a split tile's K range can be cut over
+  float *partials;      // [split tiles][max_pieces][128][32] fp32
   int *counters;        // [tiles], zero on entry and zeroed again by each tile's last arriver
   int32_t *dev_status;
   const float *a_sf32;  // NPL = 3: fp32 activation scales [M, K/16]
   const float *w_scale; // NPL = 3: fp32 weight dequantization scale (multiplies)
+  int full_per_cta;     // whole tiles per CTA: CTA c owns tiles c, c + G, ... below tile_base
+  int tile_base;        // = grid x full_per_cta; tiles from here on are split stream-K
+  int64_t rem_units;    // (tiles - tile_base) x K-steps, cut evenly over CTAs 0 .. rem_ctas - 1
+  int rem_ctas;         // min(grid, rem_units): every one of them gets at least one unit
 };
 
 // Contiguous unit range [u0, u1) of CTA c among G over U units (units = tile x K-step).
@@ -550,6 +554,35 @@ __device__ __forceinline__ void dec_range(int64_t U, int c, int G, int64_t &u0, 
 __device__ __forceinline__ int dec_owner(int64_t u, int G, int64_t U) {
   return static_cast<int>(((u + 1) * G - 1) / U);
 }
+
+// A CTA's work in order: first its contiguous slice [r, r1) of the split region's units
+// (tiles from tile_base on, each a run of num_kt K-steps), then its whole tiles c, c + G, ...
+// The split pieces come first so that their partial writes and the last arrivers' sums run
+// while the grid still streams, and every CTA ends on a whole tile (plain epilogue). Every
+// role builds the same iterator and walks the same segments.
+struct DecIter {
+  int64_t r, r1;
+  int next_full, full_left, G, num_kt, tile_base;
+  __device__ __forceinline__ bool next(int &tile, int &kb, int &ke) {
+    if (r < r1) {
+      const int64_t t = r / num_kt;
+      tile = tile_base + static_cast<int>(t);
+      kb = static_cast<int>(r - t * num_kt);
+      ke = static_cast<int>(kb + (r1 - r) < num_kt ? kb + (r1 - r) : num_kt);
+      r += ke - kb;
+      return true;
+    }
+    if (full_left > 0) {
+      tile = next_full;
+      kb = 0;
+      ke = num_kt;
+      next_full += G;
+      --full_left;
+      return true;
+    }
+    return false;
+  }
+};
 
 // AND of `v` over the `nthreads` threads of named barrier `id` (a group of warps that must
 // leave a loop together).
@@ -675,11 +708,16 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
   const int64_t k64_per_row = p.K / 64;
   float *inv_s = reinterpret_cast<float *>(smem + C::kOffSfb);  // fp32 scales: 448 / row max
   float *alpha_s = inv_s + kDecBN;                                // and rho * w_scale
-  const int64_t U = static_cast<int64_t>(p.tiles) * num_kt;
   const int G = gridDim.x;
   const int c = blockIdx.x;
-  int64_t u0, u1;
-  dec_range(U, c, G, u0, u1);
+  DecIter start;
+  start.r = start.r1 = 0;
+  if (c < p.rem_ctas) dec_range(p.rem_units, c, p.rem_ctas, start.r, start.r1);
+  start.next_full = c;
+  start.full_left = p.full_per_cta;
+  start.G = G;
+  start.num_kt = num_kt;
+  start.tile_base = p.tile_base;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -717,10 +755,9 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     }
     uint32_t it = 0;
     bool ok = true;
-    for (int64_t u = u0; u < u1 && ok;) {
-      const int tile = static_cast<int>(u / num_kt);
-      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
-      const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
+    DecIter itr = start;
+    int tile, kb, ke;
+    while (ok && itr.next(tile, kb, ke)) {
       const int64_t w0 = static_cast<int64_t>(tile) * kBM;
       for (int kt = kb; kt < ke; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
@@ -751,7 +788,6 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         }
         __syncwarp();
       }
-      u += ke - kb;
     }
     if (ok) {
       const uint32_t used = it < STAGES ? it : STAGES;
@@ -768,10 +804,9 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     if (lane == 0) {
       uint32_t it = 0, seg = 0;
       bool ok = true;
-      for (int64_t u = u0; u < u1 && ok; ++seg) {
-        const int tile = static_cast<int>(u / num_kt);
-        const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
-        const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
+      DecIter itr = start;
+      int tile, kb, ke;
+      for (; ok && itr.next(tile, kb, ke); ++seg) {
         const int buf = static_cast<int>(seg % C::kAccBufs);
         const uint32_t use = seg / C::kAccBufs;
         if (use > 0 && !mbar_wait_bounded(&acc_empty[buf], (use - 1) & 1, kWaitTimeoutNs)) {
@@ -804,7 +839,6 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         }
         if (prev >= 0) tc_commit(&empty[prev]);
         if (ok) tc_commit(&acc_full[buf]);
-        u += ke - kb;
       }
     }
     __syncwarp();
@@ -842,22 +876,30 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       pre = (ktn >= 0 && k64 < num_k64) ? __ldg(my_sf32 + k64) : make_float4(0.f, 0.f, 0.f, 0.f);
     };
     uint32_t *xbuf = reinterpret_cast<uint32_t *>(smem + C::kOffSfb + C::kOffXbuf);
-    if constexpr (NPL > 1) load_step(static_cast<int>(u0 % num_kt));
-    for (int64_t u = u0; u < u1 && ok;) {
-      const int tile = static_cast<int>(u / num_kt);
-      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
-      const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
+    DecIter itr = start;
+    int tile, kb, ke;
+    if constexpr (NPL > 1) {
+      DecIter pk = itr;
+      load_step(pk.next(tile, kb, ke) ? kb : -1);
+    }
+    while (ok && itr.next(tile, kb, ke)) {
       for (int kt = kb; kt < ke; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
         const int k64_0 = kt * kK64PerStage;
         const int nk64 = min(kK64PerStage, num_k64 - k64_0);
         // fp32 scales: split this stage's words before the wait (they need no stage data),
-        // the next stage's scales loading meanwhile (the next segment starts a tile at K = 0)
+        // the next stage's scales loading meanwhile
         uint32_t *xb = xbuf + (it & 1) * (kK64PerStage * NPL * 32);
         if constexpr (NPL > 1) {
           const float4 cur = pre;
-          load_step(kt + 1 < ke ? kt + 1 : (u + (ke - kb) < u1 ? 0 : -1));
+          int kt_next = kt + 1;
+          if (kt_next >= ke) {  // the next segment's first K-step, if any
+            DecIter pk = itr;
+            int t2, kb2, ke2;
+            kt_next = pk.next(t2, kb2, ke2) ? kb2 : -1;
+          }
+          load_step(kt_next);
           uint32_t w[NPL];
           split_scale_word<NPL>(cur, my_inv, w, bad);
 #pragma unroll
@@ -899,7 +941,6 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sf_full[stage]);
       }
-      u += ke - kb;
     }
     if (bad && p.dev_status != nullptr) atomicOr(p.dev_status, kDevErrBadScale);
   } else if (warp >= kEpiWarp0) {
@@ -918,11 +959,9 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       for (int j = 0; j < kDecBN; ++j) alpha[j] = out_alpha(p.ga, p.ga_per_row, p.gw, j, p.M);
     }
     uint32_t seg = 0;
-    for (int64_t u = u0; u < u1; ++seg) {
-      const int tile = static_cast<int>(u / num_kt);
-      const int kb = static_cast<int>(u - static_cast<int64_t>(tile) * num_kt);
-      const int ke = static_cast<int>(kb + (u1 - u) < num_kt ? kb + (u1 - u) : num_kt);
-      u += ke - kb;
+    DecIter itr = start;
+    int tile, kb, ke;
+    for (; itr.next(tile, kb, ke); ++seg) {
       const int buf = static_cast<int>(seg % C::kAccBufs);
       const uint32_t use = seg / C::kAccBufs;
       // the four epilogue warps leave together (they meet at named barriers below)
@@ -967,11 +1006,12 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         continue;
       }
       // partial tile: publish this piece, the last arriver sums the pieces in order
-      const int64_t tu0 = static_cast<int64_t>(tile) * num_kt;
-      const int first = dec_owner(tu0, G, U);
-      const int pieces = dec_owner(tu0 + num_kt - 1, G, U) - first + 1;
+      const int st = tile - p.tile_base;  // index among the split tiles
+      const int64_t tu0 = static_cast<int64_t>(st) * num_kt;
+      const int first = dec_owner(tu0, p.rem_ctas, p.rem_units);
+      const int pieces = dec_owner(tu0 + num_kt - 1, p.rem_ctas, p.rem_units) - first + 1;
       const int piece = c - first;
-      float *part_base = p.partials + static_cast<int64_t>(tile) * p.max_pieces * kBM * kDecBN;
+      float *part_base = p.partials + static_cast<int64_t>(st) * p.max_pieces * kBM * kDecBN;
       float4 *mine = reinterpret_cast<float4 *>(part_base + (static_cast<int64_t>(piece) * kBM + row) * kDecBN);
 #pragma unroll
       for (int j = 0; j < kDecBN / 4; ++j)
@@ -979,11 +1019,11 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       asm volatile("bar.sync 1, %0;" ::"n"(C::kEpiWarps * 32) : "memory");
       if (warp == kEpiWarp0 && lane == 0) {
         __threadfence();
-        const int old = atomicAdd(p.counters + tile, 1);
+        const int old = atomicAdd(p.counters + st, 1);
         *last_flag = (old == pieces - 1) ? 1 : 0;
         // the last arriver hands the counter back zeroed for the next call on this
         // workspace; a count past the pieces means the workspace was not zero on entry
-        if (old == pieces - 1) atomicExch(p.counters + tile, 0);
+        if (old == pieces - 1) atomicExch(p.counters + st, 0);
         if ((old < 0 || old >= pieces) && p.dev_status != nullptr) atomicOr(p.dev_status, kDevErrWorkspace);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(C::kEpiWarps * 32) : "memory");
@@ -1546,6 +1586,9 @@ static cudaError_t run_pair(const GemmArgs &g, int num_sms, cudaStream_t st) {
 struct DecPlan {
   int grid = 0;
   int tiles = 0;
+  int full_per_cta = 0;  // whole tiles per CTA, taken round robin from tile 0
+  int64_t rem_units = 0; // K-steps of the tiles after those, cut evenly over rem_ctas CTAs
+  int rem_ctas = 0;
   int max_pieces = 0;
   size_t partial_bytes = 0;
   bool usable = false;
@@ -1573,11 +1616,26 @@ static DecPlan dec_plan(int64_t M, int64_t N, int64_t K, int num_sms, bool sfb_f
   const int64_t U = d.tiles * num_kt;
   d.grid = static_cast<int>(U < num_sms ? U : num_sms);
   if (d.grid < 1) return d;
-  const int64_t umin = U / d.grid;  // every CTA holds at least this many units
-  int64_t mp = (num_kt - 1 + umin - 1) / umin + 1;
-  if (mp > num_kt) mp = num_kt;
-  d.max_pieces = static_cast<int>(mp);
-  d.partial_bytes = static_cast<size_t>(d.tiles) * d.max_pieces * kBM * kDecBN * sizeof(float);
+  d.full_per_cta = d.tiles / d.grid;
+  const int64_t split_tiles = d.tiles - static_cast<int64_t>(d.full_per_cta) * d.grid;
+  d.rem_units = split_tiles * num_kt;
+  // with fewer split units than CTAs only the first rem_units CTAs take one each, so that no
+  // CTA range inside a tile's K range is empty (the piece count assumes none is)
+  d.rem_ctas = static_cast<int>(d.rem_units < d.grid ? d.rem_units : d.grid);
+  if (split_tiles == 0) {
+    d.max_pieces = 1;
+    d.partial_bytes = 0;
+  } else {
+    // the most CTAs any split tile's K range meets (fewer split tiles than CTAs: a short loop)
+    auto owner = [&](int64_t u) { return ((u + 1) * d.rem_ctas - 1) / d.rem_units; };
+    int64_t mp = 1;
+    for (int64_t t = 0; t < split_tiles; ++t) {
+      const int64_t pieces = owner((t + 1) * num_kt - 1) - owner(t * num_kt) + 1;
+      if (pieces > mp) mp = pieces;
+    }
+    d.max_pieces = static_cast<int>(mp);
+    d.partial_bytes = static_cast<size_t>(split_tiles) * d.max_pieces * kBM * kDecBN * sizeof(float);
+  }
   d.usable = true;
   return d;
 }
@@ -1616,6 +1674,10 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   p.N = g.N;
   p.K = g.K;
   p.tiles = d.tiles;
+  p.full_per_cta = d.full_per_cta;
+  p.tile_base = d.full_per_cta * d.grid;
+  p.rem_units = d.rem_units;
+  p.rem_ctas = d.rem_ctas;
   p.max_pieces = d.max_pieces;
   p.counters = static_cast<int *>(g.workspace);
   p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(g.workspace) +

@@ -390,12 +390,14 @@ def test_workspace_reused_across_calls_stays_zero():
     """One zero-filled workspace serves consecutive small-M calls of different shapes (each
     against the oracle); the tiles' last arrivers hand it back zero-filled every time."""
     nv = require_cuda()
-    ws = torch.zeros(max(nv.nvfp4_gemm_workspace_bytes(32, 20480, 8192),
-                         nv.nvfp4_gemm_act_f32_workspace_bytes(40, 20480, 8192)),
-                     dtype=torch.uint8, device="cuda")
+    # (8, 19072, 1024): 149 weight tiles, so one tile is left over after a whole tile per
+    # CTA and its K-steps are cut over a few CTAs only
+    shapes = [(8, 20480, 1024), (32, 4096, 3072), (1, 20480, 8192), (17, 1032, 8192),
+              (8, 19072, 1024), (32, 4096, 3072)]
+    ws = torch.zeros(max(nv.nvfp4_gemm_workspace_bytes(*s) for s in shapes), dtype=torch.uint8,
+                     device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    for i, (M, N, K) in enumerate([(8, 20480, 1024), (32, 4096, 3072), (1, 20480, 8192),
-                                   (17, 1032, 8192), (32, 4096, 3072)]):
+    for i, (M, N, K) in enumerate(shapes):
         ops = _random_operands(M, N, K, seed=600 + i)
         _, ref = orc.gemm(*ops, want_f64=True)
         d = _to_device(nv, *ops, orc.L8x4 if i % 2 else orc.L128x4)
