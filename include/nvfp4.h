@@ -197,7 +197,8 @@ NVFP4_API int nvfp4_sf_unswizzle(const uint8_t *in, uint8_t *lin, int64_t R, int
  * M <= 32 (K <= 24576): that path splits the K range of the weight tiles evenly over the
  * SMs ("stream-K") and keeps one int arrival counter per 128-row weight tile (at the front,
  * in 16 * (workspace_bytes / 65536 + 1) bytes whatever the shape) and fp32 partial tiles
- * [tiles][pieces][128][32] after them (about 7.4 MB for N = 28672, K = 8192 on 148 SMs).
+ * [split tiles][pieces][128][32] after them (about 3.7 MB for N = 28672, K = 8192 on 148
+ * SMs: each SM owns whole weight tiles and only the tiles left over are split).
  * Pass the same workspace_bytes with a given buffer. The workspace must be zero-filled
  * before its first use (cudaMemset once); every
  * call that completes leaves the counters zero again, so it needs no per-call reset. After
@@ -262,8 +263,9 @@ NVFP4_API int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int 
  * The block-scaled MMA takes E4M3 scales only, so the kernel splits each activation row's
  * scales into three planes of E4M3 codes and one fp32 factor (rho = row maximum / 448):
  * rho * (v1 + v2 + v3) is within 2^-12 of each scale relative. One MMA per K step takes the
- * token rows once per plane (N = 96) and the epilogue adds the three fp32 partial sums. The
- * split runs inside the GEMM kernel (one launch per 32 activation rows, in stream order).
+ * token rows once per plane (N = 96) and the epilogue adds the three fp32 partial sums. Per
+ * 32 activation rows, in stream order, a small kernel splits the scales into the workspace
+ * and the GEMM kernel, launched as its programmatic dependent, streams them from there.
  * a_q      device, [M, K/2] packed E2M1, 16-byte aligned.
  * a_sf32   device, fp32 [M, K/16] row-major (the [B,1,K/16] tensor), 16-byte aligned; every
  *          scale finite and >= 0. A negative, NaN or infinite scale is an argument error the
@@ -272,7 +274,8 @@ NVFP4_API int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int 
  * w_scale  device, one fp32 (multiplies; 1 / the weight's encode scale).
  * out      device, [M, N] fp16, row-major.
  * workspace/workspace_bytes: device, 16-byte aligned, >= nvfp4_gemm_act_f32_workspace_bytes
- *          (M, N, K); same use as in nvfp4_gemm.
+ *          (M, N, K); used as in nvfp4_gemm, plus the plane words (K/64 x 384 bytes) and 32
+ *          row factors of one 32-row chunk after the partial tiles, rewritten by every call.
  * dev_status: device int32 or NULL; bit 1 a bounded wait gave up (NVFP4_ERR_TIMEOUT), bit 2
  *          a bad activation scale, bit 4 a workspace that was not zero-filled. The caller
  *          reads it after synchronizing.

@@ -492,7 +492,8 @@ struct DecCfg {
   static constexpr int kABytes = kBM * kBKBytes;                 // 16 KB of weights
   static constexpr int kBBytes = kMmaN * kBKBytes;               // 4 KB of activations a copy
   static constexpr int kSfaBytes = kK64PerStage * kSfAtomBytes;  // 2 KB of weight scales
-  static constexpr int kSfbBytes = NPL > 1 ? 0 : kK64PerStage * kSfAtomBytes;  // 128x4 atoms
+  // per stage: token scales, 128x4 atoms (E4M3 scales) or the plane words [K64][plane][32]
+  static constexpr int kSfbBytes = NPL > 1 ? kK64PerStage * NPL * 128 : kK64PerStage * kSfAtomBytes;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
   static constexpr int kOffSfa = kOffB + STAGES * kBBytes;
@@ -510,12 +511,9 @@ struct DecCfg {
   static constexpr int kEpiWarps = 4;
   static constexpr int kThreads = (kEpiWarp0 + kEpiWarps) * 32;
   static_assert(kSfCol0 + STAGES * kSlotCols <= kTmemCols, "TMEM columns");
-  // E4M3 scales: the 8x4 copy of 4 blocks of K/64 x 32 bytes. fp32 scales: 2 x 32 fp32 row
-  // factors, then the plane words of two K steps' stages, [2][kK64PerStage][NPL][32] words.
-  static constexpr int kOffXbuf = 256;
+  // E4M3 scales in 8x4: the copy of 4 blocks of K/64 x 32 bytes
   static constexpr int smem_bytes(int k64_total, bool sfb_8x4) {
-    return kOffSfb + (NPL == 1 ? (sfb_8x4 ? k64_total * 128 : 0) : kOffXbuf + 2 * kK64PerStage * NPL * 128) +
-           1024;
+    return kOffSfb + (NPL == 1 && sfb_8x4 ? k64_total * 128 : 0) + 1024;
   }
   static constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | (uint32_t(kMmaN >> 3) << 17) |
                                      (uint32_t(kBM >> 4) << 24);
@@ -536,8 +534,8 @@ struct DecParams {
   float *partials;      // [split tiles][max_pieces][128][32] fp32
   int *counters;        // [tiles], zero on entry and zeroed again by each tile's last arriver
   int32_t *dev_status;
-  const float *a_sf32;  // NPL = 3: fp32 activation scales [M, K/16]
-  const float *w_scale; // NPL = 3: fp32 weight dequantization scale (multiplies)
+  const uint32_t *planes;  // NPL = 3: plane words [K/64][NPL][32] from act_scale_planes_kernel
+  const float *row_alpha;  // NPL = 3: per-token output factors [32] from the same kernel
   int full_per_cta;     // whole tiles per CTA: CTA c owns tiles c, c + G, ... below tile_base
   int tile_base;        // = grid x full_per_cta; tiles from here on are split stream-K
   int64_t rem_units;    // (tiles - tile_base) x K-steps, cut evenly over CTAs 0 .. rem_ctas - 1
@@ -621,47 +619,6 @@ __device__ __forceinline__ float e4m3_floor(float t) {
 // scales need. A negative, NaN or infinite scale is an argument error: its block counts as
 // zero and kDevErrBadScale is ORed into the status word.
 //
-// Row factors: warp q finds the maxima of rows 8q .. 8q+7 (the loads of all eight rows in
-// flight together) and stores 448 / max and alpha = rho * w_scale per row (zero past M).
-__device__ void act_scale_row_factors(const DecParams &p, int q, int lane, float *inv_s,
-                                      float *alpha_s, int64_t k64_per_row) {
-  constexpr int kRows = 8;
-  const int groups = static_cast<int>(k64_per_row);  // 4-column groups per row (K / 64)
-  const int r0 = q * kRows;
-  const float4 *src[kRows];
-  bool live[kRows];
-#pragma unroll
-  for (int i = 0; i < kRows; ++i) {
-    live[i] = r0 + i < p.M;
-    src[i] = reinterpret_cast<const float4 *>(p.a_sf32 + (live[i] ? r0 + i : 0) * (k64_per_row * 4));
-  }
-  float mx[kRows];
-#pragma unroll
-  for (int i = 0; i < kRows; ++i) mx[i] = 0.0f;
-  for (int g = lane; g < groups; g += 32) {
-    float4 v[kRows];
-#pragma unroll
-    for (int i = 0; i < kRows; ++i) v[i] = live[i] ? __ldg(src[i] + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int i = 0; i < kRows; ++i) {
-      const float e[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (e[j] >= 0.0f && e[j] <= FLT_MAX) mx[i] = fmaxf(mx[i], e[j]);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < kRows; ++i) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
-    if (lane == 0) {
-      const bool use = live[i] && mx[i] > 0.0f;
-      inv_s[r0 + i] = use ? __fdiv_rn(448.0f, mx[i]) : 0.0f;
-      alpha_s[r0 + i] = use ? __fmul_rn(__fdiv_rn(mx[i], 448.0f), p.w_scale[0]) : 0.0f;
-    }
-  }
-}
-
 // The NPL plane words (four E4M3 codes each, one K64 step of one row) of four fp32 scales.
 template <int NPL>
 __device__ __forceinline__ void split_scale_word(float4 v, float inv, uint32_t (&w)[NPL], bool &bad) {
@@ -681,6 +638,65 @@ __device__ __forceinline__ void split_scale_word(float4 v, float inv, uint32_t (
     }
     w[NPL - 1] |= cvt_e4m3(t) << (8 * j);
   }
+}
+
+// The K-steps a CTA walks, one by one, in its segments' order (-1 once they run out).
+struct KStream {
+  DecIter itr;
+  int kt, ke;
+  __device__ __forceinline__ int next() {
+    if (kt >= ke) {
+      int tile, kb;
+      if (!itr.next(tile, kb, ke)) return -1;
+      kt = kb;
+    }
+    return kt++;
+  }
+};
+
+// The split of one chunk of up to 32 activation rows, once per call ahead of the GEMM: one
+// warp per row r finds the row maximum over its valid scales, writes the output factor
+// alpha = rho * w_scale (zero for a row past M or without a positive scale) and the NPL plane
+// words of every K64 step to planes[(k64 * NPL + plane) * 32 + r] (zero past M). It lets the
+// GEMM kernel, launched after it as a programmatic dependent, start at once: the GEMM waits
+// for this kernel only where it reads the words and factors.
+template <int NPL>
+__global__ void __launch_bounds__(32) act_scale_planes_kernel(const float *__restrict__ a_sf32, int M,
+                                                              int64_t k64_per_row,
+                                                              const float *__restrict__ w_scale,
+                                                              uint32_t *__restrict__ planes,
+                                                              float *__restrict__ row_alpha,
+                                                              int *dev_status) {
+  griddep_launch_dependents();
+  const int r = blockIdx.x;
+  const int lane = threadIdx.x;
+  const bool live = r < M;
+  const float4 *src = reinterpret_cast<const float4 *>(a_sf32 + (live ? r : 0) * (k64_per_row * 4));
+  float mx = 0.0f;
+  if (live) {
+#pragma unroll 4
+    for (int64_t g = lane; g < k64_per_row; g += 32) {
+      const float4 v = __ldg(src + g);
+      const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (e[j] >= 0.0f && e[j] <= FLT_MAX) mx = fmaxf(mx, e[j]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const bool use = live && mx > 0.0f;
+  const float inv = use ? __fdiv_rn(448.0f, mx) : 0.0f;
+  if (lane == 0) row_alpha[r] = use ? __fmul_rn(__fdiv_rn(mx, 448.0f), w_scale[0]) : 0.0f;
+  bool bad = false;
+  for (int64_t g = lane; g < k64_per_row; g += 32) {
+    const float4 v = live ? __ldg(src + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+    uint32_t w[NPL];
+    split_scale_word<NPL>(v, inv, w, bad);
+#pragma unroll
+    for (int pl = 0; pl < NPL; ++pl) planes[(g * NPL + pl) * 32 + r] = w[pl];
+  }
+  if (bad && dev_status != nullptr) atomicOr(dev_status, kDevErrBadScale);
 }
 
 template <int STAGES, int NPL>
@@ -706,8 +722,6 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
   const int num_k64 = static_cast<int>(p.K / 64);
   const int num_kt = (num_k64 + kK64PerStage - 1) / kK64PerStage;
   const int64_t k64_per_row = p.K / 64;
-  float *inv_s = reinterpret_cast<float *>(smem + C::kOffSfb);  // fp32 scales: 448 / row max
-  float *alpha_s = inv_s + kDecBN;                                // and rho * w_scale
   const int G = gridDim.x;
   const int c = blockIdx.x;
   DecIter start;
@@ -729,7 +743,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], C::kEpiWarps);
     }
-    mbar_init(sfb_ready, NPL > 1 ? 4 : 1);  // the bulk copy, or the four scale warps' split
+    mbar_init(sfb_ready, 1);  // the 8x4 copy (E4M3 activation scales)
     fence_mbar_init();
     prefetch_tmap(&tmap_w);
     prefetch_tmap(&tmap_a);
@@ -755,6 +769,26 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     }
     uint32_t it = 0;
     bool ok = true;
+    // fp32 scales: the plane words come from the kernel before this one, so the first ring
+    // pass goes out without them (its stages' byte counts include them) and, once that
+    // kernel has finished, their copies follow, before any stage can be reused
+    bool planes_out = NPL == 1;
+    auto issue_first_planes = [&](uint32_t n) {
+      if (lane == 0) {
+        griddep_wait();
+        KStream ks;
+        ks.itr = start;
+        ks.kt = ks.ke = 0;
+        for (uint32_t i = 0; i < n; ++i) {
+          const int k64 = ks.next() * kK64PerStage;
+          const int nk = min(kK64PerStage, num_k64 - k64);
+          bulk_g2s(smem + C::kOffSfbStage + i * C::kSfbBytes, p.planes + static_cast<int64_t>(k64) * NPL * 32,
+                   nk * NPL * 128, &full[i]);
+        }
+      }
+      __syncwarp();
+      planes_out = true;
+    };
     DecIter itr = start;
     int tile, kb, ke;
     while (ok && itr.next(tile, kb, ke)) {
@@ -762,6 +796,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       for (int kt = kb; kt < ke; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
+        if (!planes_out && it == STAGES) issue_first_planes(STAGES);
         if (it >= STAGES && !mbar_wait_warp(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
@@ -770,7 +805,8 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         const int k64_0 = kt * kK64PerStage;
         const int nk64 = min(kK64PerStage, num_k64 - k64_0);
         if (lane == 0) {
-          const uint32_t sf_bytes = (p.a_sf_8x4 ? 1 : 2) * nk64 * kSfAtomBytes;
+          const uint32_t sf_bytes =
+              nk64 * kSfAtomBytes + (NPL > 1 ? nk64 * NPL * 128 : p.a_sf_8x4 ? 0 : nk64 * kSfAtomBytes);
           mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + sf_bytes);
           tma_load_2d(smem + C::kOffA + stage * C::kABytes, &tmap_w, kt * kBKBytes,
                       static_cast<int32_t>(w0), &full[stage]);
@@ -781,14 +817,20 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
           bulk_g2s(smem + C::kOffSfa + stage * C::kSfaBytes,
                    p.w_sf + ((w0 / 128) * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
                    &full[stage]);
-          if (!p.a_sf_8x4)  // tokens 0..31 sit in the first 128-row block of the 128x4 scales
+          if (NPL > 1) {
+            if (planes_out)
+              bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
+                       p.planes + static_cast<int64_t>(k64_0) * NPL * 32, nk64 * NPL * 128, &full[stage]);
+          } else if (!p.a_sf_8x4) {  // tokens 0..31: the first 128-row block of the 128x4 scales
             bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
                      p.a_sf + static_cast<int64_t>(k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
                      &full[stage]);
+          }
         }
         __syncwarp();
       }
     }
+    if (!planes_out) issue_first_planes(it < STAGES ? it : STAGES);
     if (ok) {
       const uint32_t used = it < STAGES ? it : STAGES;
       for (uint32_t i = 0; i < used; ++i) {
@@ -848,68 +890,21 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t it = 0;
     bool ok = true;
-    if constexpr (NPL > 1) {
-      act_scale_row_factors(p, q, lane, inv_s, alpha_s, k64_per_row);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sfb_ready);
-    }
     if (p.a_sf_8x4 && !mbar_wait_warp(sfb_ready, 0, kWaitTimeoutNs)) {
       if (lane == 0) report_timeout(p.dev_status);
       ok = false;
     }
-    if constexpr (NPL > 1) ok = group_all(ok, 2, 128);  // the scale warps enter the loop together
     // token `lane`'s 8x4 words: block lane / 8, byte (lane % 8) * 4 of each 32-byte step
     const uint8_t *my8x4 = sfb_8x4 + (lane / 8) * (k64_per_row * 32) + (lane % 8) * 4;
-    // fp32 scales: token `lane`'s row and factor (a token past M reads row 0 with factor 0)
-    const float4 *my_sf32 = nullptr;
-    float my_inv = 0.0f;
-    bool bad = false;
-    if constexpr (NPL > 1) {
-      my_sf32 = reinterpret_cast<const float4 *>(p.a_sf32 + (lane < p.M ? lane : 0) * (k64_per_row * 4));
-      my_inv = ok ? inv_s[lane] : 0.0f;
-    }
-    // warp q splits K64 step q of each stage (token `lane`'s four fp32 scales, loaded one
-    // stage ahead) and the four warps exchange the plane words through shared memory
-    float4 pre = make_float4(0.f, 0.f, 0.f, 0.f);
-    auto load_step = [&](int ktn) {
-      const int k64 = ktn * kK64PerStage + q;
-      pre = (ktn >= 0 && k64 < num_k64) ? __ldg(my_sf32 + k64) : make_float4(0.f, 0.f, 0.f, 0.f);
-    };
-    uint32_t *xbuf = reinterpret_cast<uint32_t *>(smem + C::kOffSfb + C::kOffXbuf);
     DecIter itr = start;
     int tile, kb, ke;
-    if constexpr (NPL > 1) {
-      DecIter pk = itr;
-      load_step(pk.next(tile, kb, ke) ? kb : -1);
-    }
     while (ok && itr.next(tile, kb, ke)) {
       for (int kt = kb; kt < ke; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
         const int k64_0 = kt * kK64PerStage;
         const int nk64 = min(kK64PerStage, num_k64 - k64_0);
-        // fp32 scales: split this stage's words before the wait (they need no stage data),
-        // the next stage's scales loading meanwhile
-        uint32_t *xb = xbuf + (it & 1) * (kK64PerStage * NPL * 32);
-        if constexpr (NPL > 1) {
-          const float4 cur = pre;
-          int kt_next = kt + 1;
-          if (kt_next >= ke) {  // the next segment's first K-step, if any
-            DecIter pk = itr;
-            int t2, kb2, ke2;
-            kt_next = pk.next(t2, kb2, ke2) ? kb2 : -1;
-          }
-          load_step(kt_next);
-          uint32_t w[NPL];
-          split_scale_word<NPL>(cur, my_inv, w, bad);
-#pragma unroll
-          for (int pl = 0; pl < NPL; ++pl) xb[(q * NPL + pl) * 32 + lane] = w[pl];
-        }
-        bool got = mbar_wait_warp(&full[stage], round & 1, kWaitTimeoutNs);
-        // the four scale warps agree (and publish their words) before any leaves or reads:
-        // a buffer is rewritten two stages later, after every warp passed the next agreement
-        if constexpr (NPL > 1) got = group_all(got, 2, 128);
-        if (!got) {
+        if (!mbar_wait_warp(&full[stage], round & 1, kWaitTimeoutNs)) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
           break;
@@ -923,10 +918,11 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
           const uint32_t wa =
               *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
           tmem_st_x1(slot + a * 4 + q, wa);  // quarter q reads column base + q
-          if constexpr (NPL > 1) {
+          if constexpr (NPL > 1) {  // plane p's words to column p of the step
+            const uint8_t *sB = smem + C::kOffSfbStage + stage * C::kSfbBytes + a * (NPL * 128) + lane * 4;
 #pragma unroll
             for (int pl = 0; pl < NPL; ++pl)
-              tmem_st_x1(slot + kK64PerStage * 4 + a * 4 + pl, xb[(a * NPL + pl) * 32 + lane]);
+              tmem_st_x1(slot + kK64PerStage * 4 + a * 4 + pl, *reinterpret_cast<const uint32_t *>(sB + pl * 128));
           } else if (p.a_sf_8x4) {
             tmem_st_x1(slot + kK64PerStage * 4 + a * 4,
                        *reinterpret_cast<const uint32_t *>(my8x4 + (k64_0 + a) * 32));
@@ -942,18 +938,15 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         if (lane == 0) mbar_arrive(&sf_full[stage]);
       }
     }
-    if (bad && p.dev_status != nullptr) atomicOr(p.dev_status, kDevErrBadScale);
   } else if (warp >= kEpiWarp0) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;  // weight row within the tile (accumulator lane)
     float alpha[kDecBN];  // per token (accumulator column)
     if constexpr (NPL > 1) {
-      // the row factors come from the scale warps (zero if they never arrived: the
-      // accumulator waits below then give up too)
-      const bool got = mbar_wait_warp(sfb_ready, 0, kWaitTimeoutNs);
+      griddep_wait();  // the row factors come from the kernel before this one
 #pragma unroll
-      for (int j = 0; j < kDecBN; ++j) alpha[j] = got ? alpha_s[j] : 0.0f;
+      for (int j = 0; j < kDecBN; ++j) alpha[j] = __ldcg(p.row_alpha + j);
     } else {
 #pragma unroll
       for (int j = 0; j < kDecBN; ++j) alpha[j] = out_alpha(p.ga, p.ga_per_row, p.gw, j, p.M);
@@ -1647,9 +1640,16 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   return d.usable ? workspace_for(d.partial_bytes) : 0;
 }
 
+// fp32 activation scales: after the partial tiles, the plane words of one 32-row chunk
+// ([K/64][3][32] words) and its 32 row factors.
+static constexpr int kActPlanes = 3;
+static size_t act_planes_bytes(int64_t K) {
+  return static_cast<size_t>(K / 64) * kActPlanes * 128 + kDecBN * sizeof(float);
+}
+
 size_t gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
   const DecPlan d = dec_plan(M < kDecBN ? M : kDecBN, N, K, num_sms);
-  return d.usable ? workspace_for(d.partial_bytes) : 0;
+  return d.usable ? workspace_for(d.partial_bytes + act_planes_bytes(K)) : 0;
 }
 
 template <int STAGES, int NPL = 1>
@@ -1662,10 +1662,8 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   DecParams p{};
   p.w_sf = g.w_sf;
   p.a_sf = g.a_sf;
-  p.a_sf_8x4 = (NPL > 1 || g.a_layout == kSf8x4) ? 1 : 0;
-  p.a_sf_rows = NPL > 1 ? kDecBN : p.a_sf_8x4 ? (g.M + 7) / 8 * 8 : (g.M + 127) / 128 * 128;
-  p.a_sf32 = g.a_sf32;
-  p.w_scale = g.w_scale;
+  p.a_sf_8x4 = (NPL == 1 && g.a_layout == kSf8x4) ? 1 : 0;
+  p.a_sf_rows = p.a_sf_8x4 ? (g.M + 7) / 8 * 8 : (g.M + 127) / 128 * 128;
   p.ga = g.a_g;
   p.gw = g.w_g;
   p.ga_per_row = g.a_g_per_row;
@@ -1687,15 +1685,39 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   const int smem = C::smem_bytes(static_cast<int>(g.K / 64), p.a_sf_8x4 != 0);
   e = ensure_smem_attr(gemm_nvfp4_decode_kernel<STAGES, NPL>, smem);
   if (e != cudaSuccess) return e;
-  gemm_nvfp4_decode_kernel<STAGES, NPL><<<d.grid, C::kThreads, smem, st>>>(mw, ma, p);
-  return cudaGetLastError();
+  if constexpr (NPL == 1) {
+    gemm_nvfp4_decode_kernel<STAGES, NPL><<<d.grid, C::kThreads, smem, st>>>(mw, ma, p);
+    return cudaGetLastError();
+  } else {
+    // the split kernel first (one warp per row); the GEMM may start while it runs and waits
+    // for it only where it reads the words and factors (griddepcontrol)
+    uint8_t *planes = static_cast<uint8_t *>(g.workspace) + counter_region(g.workspace_bytes) + d.partial_bytes;
+    p.planes = reinterpret_cast<const uint32_t *>(planes);
+    p.row_alpha = reinterpret_cast<const float *>(planes + static_cast<size_t>(g.K / 64) * NPL * 128);
+    act_scale_planes_kernel<NPL><<<kDecBN, 32, 0, st>>>(g.a_sf32, static_cast<int>(g.M), g.K / 64, g.w_scale,
+                                                         reinterpret_cast<uint32_t *>(planes),
+                                                         const_cast<float *>(p.row_alpha), g.dev_status);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(d.grid);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_nvfp4_decode_kernel<STAGES, NPL>, mw, ma, p);
+  }
 }
 
 bool gemm_act_f32_supported(int64_t K) { return K / 2 <= (int64_t(1) << 31); }
 
-// The GEMM with fp32 activation scales: the small-M stream-K kernel with three scale planes,
-// once per 32 activation rows (the rows of a chunk are independent; the chunks run in stream
-// order and share the workspace).
+// The GEMM with fp32 activation scales: per 32 activation rows, the split kernel and the
+// small-M stream-K kernel with three scale planes (the rows of a chunk are independent; the
+// chunks run in stream order and share the workspace).
 cudaError_t launch_gemm_act_f32(const GemmArgs &g, int num_sms, cudaStream_t st) {
   for (int64_t m0 = 0; m0 < g.M; m0 += kDecBN) {
     GemmArgs c = g;
@@ -1705,7 +1727,7 @@ cudaError_t launch_gemm_act_f32(const GemmArgs &g, int num_sms, cudaStream_t st)
     c.out = static_cast<__half *>(g.out) + m0 * g.N;
     const DecPlan d = dec_plan(c.M, g.N, g.K, num_sms);
     if (!d.usable) return cudaErrorNotSupported;
-    const cudaError_t e = run_decode<7, 3>(c, d, st);
+    const cudaError_t e = run_decode<7, kActPlanes>(c, d, st);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
