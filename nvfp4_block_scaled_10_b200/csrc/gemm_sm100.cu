@@ -534,7 +534,7 @@ struct DecParams {
   float *partials;      // [split tiles][max_pieces][128][32] fp32
   int *counters;        // [tiles], zero on entry and zeroed again by each tile's last arriver
   int32_t *dev_status;
-  const uint32_t *planes;  // NPL = 3: plane words [K/64][NPL][32] from act_scale_planes_kernel
+  const uint32_t *planes;  // NPL = 3: plane words [K/64][NPL][32] (launch_act_scale_planes)
   const float *row_alpha;  // NPL = 3: per-token output factors [32] from the same kernel
   int full_per_cta;     // whole tiles per CTA: CTA c owns tiles c, c + G, ... below tile_base
   int tile_base;        // = grid x full_per_cta; tiles from here on are split stream-K
@@ -601,45 +601,6 @@ __device__ __forceinline__ bool group_all(bool v, int id, int nthreads) {
 __device__ __forceinline__ bool epi_all(bool v, int nthreads) { return group_all(v, 1, nthreads); }
 
 
-// The largest E4M3 value <= t, for 0 <= t <= 448 (as an fp32 value). Every E4M3 value is
-// k * 2^E with an integer 0 <= k <= 15, so cutting t to four significant bits (normal range,
-// t >= 2^-6) or to a multiple of 2^-9 (subnormal range) lands on one, and t minus it is exact.
-__device__ __forceinline__ float e4m3_floor(float t) {
-  if (t >= 0x1p-6f) return __uint_as_float(__float_as_uint(t) & 0xFFF00000u);
-  return __fmul_rn(floorf(__fmul_rn(t, 512.0f)), 0x1p-9f);
-}
-
-// fp32 activation scales ("Fused Nvfp4 GEMM All Reduce Plugin": a combined FP32 scale
-// [B,1,K/16] per activation block, which the block-scaled MMA cannot take) become NPL planes of
-// E4M3 codes and one fp32 factor per row: with rho = max_c sa[r,c] / 448 and t = sa * (448 /
-// max) <= 448, plane 1 holds floor_E4M3(t), plane 2 floor_E4M3 of the exact remainder, plane 3
-// the remainder rounded to nearest. Each floor keeps at least four significant bits, so
-// rho * (v1 + v2 + v3) is within 2^-12 of sa relative (blocks below 2^-6 / 448 of the row
-// maximum within 2^-10 * rho absolute), and all codes are non-negative, as the MMA's unsigned
-// scales need. A negative, NaN or infinite scale is an argument error: its block counts as
-// zero and kDevErrBadScale is ORed into the status word.
-//
-// The NPL plane words (four E4M3 codes each, one K64 step of one row) of four fp32 scales.
-template <int NPL>
-__device__ __forceinline__ void split_scale_word(float4 v, float inv, uint32_t (&w)[NPL], bool &bad) {
-  const float e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int pl = 0; pl < NPL; ++pl) w[pl] = 0u;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const bool ok = e[j] >= 0.0f && e[j] <= FLT_MAX;
-    bad |= !ok;
-    float t = ok ? fminf(__fmul_rn(e[j], inv), 448.0f) : 0.0f;
-#pragma unroll
-    for (int pl = 0; pl + 1 < NPL; ++pl) {
-      const float f = e4m3_floor(t);
-      w[pl] |= cvt_e4m3(f) << (8 * j);
-      t = __fsub_rn(t, f);
-    }
-    w[NPL - 1] |= cvt_e4m3(t) << (8 * j);
-  }
-}
-
 // The K-steps a CTA walks, one by one, in its segments' order (-1 once they run out).
 struct KStream {
   DecIter itr;
@@ -653,51 +614,6 @@ struct KStream {
     return kt++;
   }
 };
-
-// The split of one chunk of up to 32 activation rows, once per call ahead of the GEMM: one
-// warp per row r finds the row maximum over its valid scales, writes the output factor
-// alpha = rho * w_scale (zero for a row past M or without a positive scale) and the NPL plane
-// words of every K64 step to planes[(k64 * NPL + plane) * 32 + r] (zero past M). It lets the
-// GEMM kernel, launched after it as a programmatic dependent, start at once: the GEMM waits
-// for this kernel only where it reads the words and factors.
-template <int NPL>
-__global__ void __launch_bounds__(32) act_scale_planes_kernel(const float *__restrict__ a_sf32, int M,
-                                                              int64_t k64_per_row,
-                                                              const float *__restrict__ w_scale,
-                                                              uint32_t *__restrict__ planes,
-                                                              float *__restrict__ row_alpha,
-                                                              int *dev_status) {
-  griddep_launch_dependents();
-  const int r = blockIdx.x;
-  const int lane = threadIdx.x;
-  const bool live = r < M;
-  const float4 *src = reinterpret_cast<const float4 *>(a_sf32 + (live ? r : 0) * (k64_per_row * 4));
-  float mx = 0.0f;
-  if (live) {
-#pragma unroll 4
-    for (int64_t g = lane; g < k64_per_row; g += 32) {
-      const float4 v = __ldg(src + g);
-      const float e[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if (e[j] >= 0.0f && e[j] <= FLT_MAX) mx = fmaxf(mx, e[j]);
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const bool use = live && mx > 0.0f;
-  const float inv = use ? __fdiv_rn(448.0f, mx) : 0.0f;
-  if (lane == 0) row_alpha[r] = use ? __fmul_rn(__fdiv_rn(mx, 448.0f), w_scale[0]) : 0.0f;
-  bool bad = false;
-  for (int64_t g = lane; g < k64_per_row; g += 32) {
-    const float4 v = live ? __ldg(src + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-    uint32_t w[NPL];
-    split_scale_word<NPL>(v, inv, w, bad);
-#pragma unroll
-    for (int pl = 0; pl < NPL; ++pl) planes[(g * NPL + pl) * 32 + r] = w[pl];
-  }
-  if (bad && dev_status != nullptr) atomicOr(dev_status, kDevErrBadScale);
-}
 
 template <int STAGES, int NPL>
 __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
@@ -1642,7 +1558,6 @@ size_t gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int num_sms) {
 
 // fp32 activation scales: after the partial tiles, the plane words of one 32-row chunk
 // ([K/64][3][32] words) and its 32 row factors.
-static constexpr int kActPlanes = 3;
 static size_t act_planes_bytes(int64_t K) {
   return static_cast<size_t>(K / 64) * kActPlanes * 128 + kDecBN * sizeof(float);
 }
@@ -1694,10 +1609,9 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
     uint8_t *planes = static_cast<uint8_t *>(g.workspace) + counter_region(g.workspace_bytes) + d.partial_bytes;
     p.planes = reinterpret_cast<const uint32_t *>(planes);
     p.row_alpha = reinterpret_cast<const float *>(planes + static_cast<size_t>(g.K / 64) * NPL * 128);
-    act_scale_planes_kernel<NPL><<<kDecBN, 32, 0, st>>>(g.a_sf32, static_cast<int>(g.M), g.K / 64, g.w_scale,
-                                                         reinterpret_cast<uint32_t *>(planes),
-                                                         const_cast<float *>(p.row_alpha), g.dev_status);
-    e = cudaGetLastError();
+    static_assert(NPL == kActPlanes, "the split kernel writes kActPlanes planes");
+    e = launch_act_scale_planes(g.a_sf32, g.M, g.K, g.w_scale, reinterpret_cast<uint32_t *>(planes),
+                                const_cast<float *>(p.row_alpha), g.dev_status, st);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(d.grid);

@@ -36,6 +36,16 @@ cudaError_t launch_sf_swizzle(const uint8_t *lin, uint8_t *out, int64_t R, int64
 cudaError_t launch_sf_unswizzle(const uint8_t *in, uint8_t *lin, int64_t R, int64_t C, int layout,
                                 int64_t Cp, int num_sms, cudaStream_t st);
 
+// act_planes.cu: the fp32 activation scales of up to 32 rows [M, K/16] become kActPlanes
+// planes of E4M3 words planes[(k64 * kActPlanes + plane) * 32 + row] and per-row output
+// factors row_alpha[32] (= row maximum / 448 * w_scale; zero past M). Bad scales OR
+// kDevErrBadScale into dev_status. Written for the GEMM launched next, which may start early
+// (programmatic dependent launch) and waits for this kernel where it reads them.
+constexpr int kActPlanes = 3;
+cudaError_t launch_act_scale_planes(const float *a_sf32, int64_t M, int64_t K, const float *w_scale,
+                                    uint32_t *planes, float *row_alpha, int *dev_status,
+                                    cudaStream_t st);
+
 // gemm_sm100.cu
 struct GemmArgs {
   const uint8_t *a_q;
