@@ -597,7 +597,7 @@ __device__ __forceinline__ bool group_all(bool v, int id, int nthreads) {
   return r != 0;
 }
 
-// Named barrier 1: the epilogue warps; 2: the scale warps.
+// Named barrier 1: the epilogue warps.
 __device__ __forceinline__ bool epi_all(bool v, int nthreads) { return group_all(v, 1, nthreads); }
 
 

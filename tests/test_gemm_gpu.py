@@ -226,8 +226,9 @@ def _run_act_f32(nv, a, sa32, w, sw, w_scale):
     return out.cpu().view(torch.int16).numpy().view(np.uint16), status.item()
 
 
-# M <= 32 one launch; M > 32 one launch per 32 rows (ragged last chunk); K = 64 a single MMA
-# K step; K up to 32768 (the scales are split per pipeline stage, so K has no limit).
+# M <= 32 one split kernel and one GEMM launch; M > 32 that pair per 32 rows (ragged last
+# chunk); K = 64 a single MMA K step; K up to 32768 (the plane words live in the workspace,
+# so K has no shared-memory limit).
 ACT_F32 = [(1, 256, 512), (5, 136, 64), (32, 512, 1024), (33, 256, 512), (80, 1032, 2048),
            (17, 1032, 8192), (8, 264, 16384), (2, 520, 32768)]
 
