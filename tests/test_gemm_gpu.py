@@ -287,6 +287,45 @@ def test_gemm_act_f32_bad_scales_flagged():
     gemm_close(got, ref)
 
 
+def test_gemm_act_f32_graph_replay_matches_eager():
+    """The split kernel and the GEMM it launches as a programmatic dependent, captured in a
+    CUDA graph (two 32-row chunks, so four kernels): every replay, with new activation
+    scales copied in between, equals an eager call bit for bit and the oracle."""
+    nv = require_cuda()
+    M, N, K = 40, 1032, 2048
+    a = workloads.random_bytes((M, K // 2), 901)
+    w = workloads.random_bytes((N, K // 2), 902)
+    sw = workloads.random_bytes((N, K // 16), 903, 0x28, 0x48)
+    w_scale = float(np.float32(1.0 / 250.0))
+    sets = [_act_f32_scales(kind, M, K, 904 + i) for i, kind in enumerate(["product", "wide"])]
+    a_d, w_d = torch.from_numpy(a).cuda(), torch.from_numpy(w).cuda()
+    sw_d = torch.from_numpy(orc.swizzle(sw, orc.L128x4)).cuda()
+    wsc = torch.tensor([w_scale], dtype=torch.float32, device="cuda")
+    sa_d = torch.from_numpy(np.ascontiguousarray(sets[0])).cuda()
+    out = torch.empty(M, N, dtype=torch.float16, device="cuda")
+    ws = torch.zeros(nv.nvfp4_gemm_act_f32_workspace_bytes(M, N, K), dtype=torch.uint8, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        nv.nvfp4_gemm_act_f32(a_d, sa_d, w_d, sw_d, wsc, out=out, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        nv.nvfp4_gemm_act_f32(a_d, sa_d, w_d, sw_d, wsc, out=out, workspace=ws, dev_status=status)
+    for sa in sets + sets[:1]:
+        sa_d.copy_(torch.from_numpy(np.ascontiguousarray(sa)))
+        graph.replay()
+        torch.cuda.synchronize()
+        replayed = out.cpu().view(torch.int16).numpy().view(np.uint16).copy()
+        eager = nv.nvfp4_gemm_act_f32(a_d, sa_d, w_d, sw_d, wsc, workspace=ws, dev_status=status)
+        torch.cuda.synchronize()
+        assert np.array_equal(replayed, eager.cpu().view(torch.int16).numpy().view(np.uint16))
+        _, ref = orc.gemm_act_f32(a, sa, w, sw, w_scale, want_f64=True)
+        gemm_close(replayed, ref)
+    assert status.item() == 0
+    del graph
+
+
 @pytest.mark.parametrize("M", [1, 32])
 def test_gemm_act_f32_decode_workload(decode_weights, M):
     """The decode workload (W NVFP4 [28672, 8192]) under the fp32 activation contract: the
