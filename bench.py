@@ -203,6 +203,33 @@ def job_throughput(world, units_per_rank_step, ms_per_step):
 
 # ----------------------------------------------------------------------------- our arm
 
+def workload_config(wl, args):
+    """The workload keys of the JSON line's config (shared by both arms)."""
+    if wl == "per_token":
+        return {"workload": "per-token NVFP4 quantize", "shape": [8192, 7168], "input": "bf16",
+                "dist": "N(0,1), 0.1% of entries x50", "scales": "E4M3 128x4",
+                "global_scale": "fp32 per token", "l2": "input rotated over 3 copies (352 MB > 126 MB L2)"}
+    if wl == "swiglu":
+        return {"workload": "fused SwiGLU + NVFP4 quantize", "shape": [4096, 2 * 14336],
+                "input": "bf16", "dist": "N(0,1)", "scales": "E4M3 128x4",
+                "global_scale": "fp32 per tensor", "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
+    if wl == "swiglu_fp8":
+        return {"workload": "fused SwiGLU + FP8 E4M3 quantize", "shape": [4096, 2 * 14336],
+                "input": "bf16", "dist": "N(0,1)", "output": "E4M3 [M, H], scale 448/60",
+                "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
+    if wl in ("decode", "decode_f32"):
+        M, N, K, ncopy = args.m, 28672, 8192, 2
+    elif wl == "prefill":
+        M, N, K, ncopy = 8192, 8192, 8192, 3
+    elif wl == "tiny":
+        M, N, K, ncopy = 16, 256, 512, 1
+    else:
+        raise SystemExit(f"unknown workload {wl}")
+    return {"workload": f"NVFP4 GEMM ({wl})", "M": M, "N": N, "K": K,
+            "a_scales": "fp32 [M, K/16]" if wl == "decode_f32" else args.a_layout,
+            "w_scales": "128x4", "out": "fp16", "l2": f"operands rotated over {ncopy} copies"}
+
+
 def run_ours(args, rank, world, torch, dist):
     import nvfp4_block_scaled_10_b200 as nv
     from nvfp4_block_scaled_10_b200 import build, workloads
@@ -230,9 +257,7 @@ def run_ours(args, rank, world, torch, dist):
         def step(i):
             nv.nvfp4_quantize(copies[i % 3], g, per_token=True, sf_layout=nv.SF_128x4, q=q, sf=sf)
         launches_per_step, period = 1, 3
-        workload_desc = {"workload": "per-token NVFP4 quantize", "shape": [M, K], "input": "bf16",
-                         "dist": "N(0,1), 0.1% of entries x50", "scales": "E4M3 128x4",
-                         "global_scale": "fp32 per token", "l2": "input rotated over 3 copies (352 MB > 126 MB L2)"}
+        workload_desc = workload_config(wl, args)
         unit, factor = "GB/s", alg["bytes"] / 1e9
     elif wl == "swiglu":
         M, H = 4096, 14336
@@ -248,9 +273,7 @@ def run_ours(args, rank, world, torch, dist):
         def step(i):
             nv.swiglu_nvfp4_quantize(copies[i % 2], gdev, sf_layout=nv.SF_128x4, q=q, sf=sf)
         launches_per_step, period = 1, 2
-        workload_desc = {"workload": "fused SwiGLU + NVFP4 quantize", "shape": [M, 2 * H],
-                         "input": "bf16", "dist": "N(0,1)", "scales": "E4M3 128x4",
-                         "global_scale": "fp32 per tensor", "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
+        workload_desc = workload_config(wl, args)
         unit, factor = "GB/s", alg["bytes"] / 1e9
     elif wl == "swiglu_fp8":
         M, H = 4096, 14336
@@ -265,9 +288,7 @@ def run_ours(args, rank, world, torch, dist):
         def step(i):
             nv.swiglu_fp8_quantize(copies[i % 2], sdev, q=q)
         launches_per_step, period = 1, 2
-        workload_desc = {"workload": "fused SwiGLU + FP8 E4M3 quantize", "shape": [M, 2 * H],
-                         "input": "bf16", "dist": "N(0,1)", "output": "E4M3 [M, H], scale 448/60",
-                         "l2": "input rotated over 2 copies (470 MB > 126 MB L2)"}
+        workload_desc = workload_config(wl, args)
         unit, factor = "GB/s", alg["bytes"] / 1e9
     elif wl in ("decode", "prefill", "tiny", "decode_f32"):
         if wl in ("decode", "decode_f32"):
@@ -325,10 +346,8 @@ def run_ours(args, rank, world, torch, dist):
             kernels_per_step = 2 * ((M + 31) // 32)
             launch_scope = ("the split kernel act_scale_planes_kernel<3> and the GEMM together "
                             "(one graph step; the GEMM alone is shorter)")
-        workload_desc = {"workload": f"NVFP4 GEMM ({wl})", "M": M, "N": N, "K": K,
-                         "a_scales": "fp32 [M, K/16]" if wl == "decode_f32" else args.a_layout,
-                         "w_scales": "128x4", "out": "fp16",
-                         "l2": f"operands rotated over {ncopy} copies"}
+        workload_desc = workload_config(wl, args)
+        assert (workload_desc["M"], workload_desc["N"], workload_desc["K"]) == (M, N, K)
         if wl in ("decode", "decode_f32"):
             unit, factor = "GB/s", alg["bytes"] / 1e9
         else:
@@ -645,7 +664,8 @@ def run_reference(args, rank, world):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
-            "config": {"workload": args.workload, "sample": desc, "runs": "CPU oracle (plain C)"},
+            "config": {**workload_config(args.workload, args), "parallelism": f"replicas x{world}",
+                       "sample": desc, "runs": "CPU oracle (plain C)"},
             "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
