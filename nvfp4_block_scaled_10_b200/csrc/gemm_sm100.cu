@@ -470,20 +470,21 @@ __global__ void __launch_bounds__(Cfg<BN, STAGES, SWAP>::kThreads, 1)
 
 // Small-M (decode) form, M <= 32: the operands swap roles (128 weight rows are the MMA's A
 // operand, the <= 32 tokens its N = 32 columns) and the work is split evenly over a resident
-// grid by K-steps ("stream-K"): the tiles x K-steps units are cut into one contiguous range
-// per CTA, so every CTA streams the same amount of weight bytes whatever the tile count.
-// A CTA whose range covers only part of a tile's K writes its fp32 partial accumulator to
-// the workspace; the last CTA to finish a tile (a per-tile arrival counter) adds the pieces
-// in piece order (deterministic), writes the fp16 result and zeroes the counter again, so a
-// workspace zero-filled once stays ready for the next call with no memset node per call. Activation scales: with the
-// 8x4 layout the <= 32 rows of all K (K/16 bytes each, four contiguous 8-row blocks) are
-// copied into shared memory once per CTA; with the 128x4 layout the activation atoms of
-// each ring stage are copied with the weight atoms.
+// grid of G CTAs ("stream-K"). CTA c owns the whole weight tiles c, c + G, ...; the K-steps
+// of the tiles left over are cut into one contiguous slice per CTA, which it runs first, so
+// every CTA streams the same amount of weight bytes whatever the tile count and ends on a
+// whole tile. A CTA whose slice covers only part of a tile's K writes its fp32 partial
+// accumulator to the workspace; the last CTA to finish such a tile (a per-tile arrival
+// counter) adds the pieces in piece order (deterministic), writes the fp16 result and zeroes
+// the counter again, so a workspace zero-filled once stays ready for the next call with no
+// memset node per call. Activation scales: with the 8x4 layout the <= 32 rows of all K (K/16
+// bytes each, four contiguous 8-row blocks) are copied into shared memory once per CTA; with
+// the 128x4 layout the activation atoms of each ring stage are copied with the weight atoms.
 constexpr int kDecBN = 32;
 constexpr int kDecMaxSfbBytes = 48 * 1024;  // preloaded activation scales: K <= 24576
 
 // NPL = 1: E4M3 activation scales. NPL = 3: fp32 activation scales split per row into three
-// planes of E4M3 codes (see split_act_scales). The MMA's N operand then holds the 32 token
+// planes of E4M3 codes (act_planes.cu), copied with each ring stage. The MMA's N operand then holds the 32 token
 // rows three times (rows 32 p + j = token j under plane p's scales), one N = 96 MMA per K step
 // makes three partial sums per token, and the epilogue adds them.
 template <int STAGES, int NPL = 1>
@@ -1606,12 +1607,13 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   } else {
     // the split kernel first (one warp per row); the GEMM may start while it runs and waits
     // for it only where it reads the words and factors (griddepcontrol)
-    uint8_t *planes = static_cast<uint8_t *>(g.workspace) + counter_region(g.workspace_bytes) + d.partial_bytes;
-    p.planes = reinterpret_cast<const uint32_t *>(planes);
-    p.row_alpha = reinterpret_cast<const float *>(planes + static_cast<size_t>(g.K / 64) * NPL * 128);
     static_assert(NPL == kActPlanes, "the split kernel writes kActPlanes planes");
-    e = launch_act_scale_planes(g.a_sf32, g.M, g.K, g.w_scale, reinterpret_cast<uint32_t *>(planes),
-                                const_cast<float *>(p.row_alpha), g.dev_status, st);
+    uint8_t *region = static_cast<uint8_t *>(g.workspace) + counter_region(g.workspace_bytes) + d.partial_bytes;
+    uint32_t *planes = reinterpret_cast<uint32_t *>(region);
+    float *row_alpha = reinterpret_cast<float *>(region + static_cast<size_t>(g.K / 64) * NPL * 128);
+    p.planes = planes;
+    p.row_alpha = row_alpha;
+    e = launch_act_scale_planes(g.a_sf32, g.M, g.K, g.w_scale, planes, row_alpha, g.dev_status, st);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(d.grid);
