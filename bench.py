@@ -3,6 +3,7 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload per_token|swiglu|swiglu_fp8|decode|decode_f32|prefill|tiny]
                     [--m 32] [--a-layout 128x4|8x4] [--no-cpu-baseline] [--no-all-cores]
+                    [--cpu-seconds 10]
 
 Default workload: per-token NVFP4 quantize of X bf16 [8192, 7168] (N(0,1) with 0.1% of
 entries x50), one fp32 global scale per token, E4M3 scales in the 128x4 layout. A step is
@@ -10,10 +11,12 @@ one call of the path on one batch; inputs are resident in HBM and rotated over e
 copies that no step finds its input in the 126 MB L2.
 
 Prints one JSON line (rank 0). `value` is whole-job throughput in the workload's unit
-(GB/s of algorithmic bytes for the quantize kernels, TFLOP/s for the GEMMs), measured with
+(GB/s of algorithmic bytes for the quantize kernels and the decode GEMMs, TFLOP/s for the
+prefill and tiny GEMMs), measured with
 CUDA events on the launching stream, max over ranks. Multi-GPU runs are independent
 replicas (weak scaling): the path has no exchange step. `cpu_baseline` times the oracle on
-a bounded sample on one host core and, under `all_cores`, on every host core.
+a bounded sample on one host core, repeated for about --cpu-seconds, and, under
+`all_cores`, on every host core.
 """
 from __future__ import annotations
 
@@ -635,12 +638,17 @@ def cpu_baseline(wl, args):
 
     oracle.lib()  # build check and library load stay out of the timing
     fn, units, desc, unit = _oracle_sample(wl, args)
-    t = time.perf_counter()
-    fn()
-    dt = time.perf_counter() - t
+    # repeat the sample until about args.cpu_seconds of CPU work have run
+    reps, t = 0, time.perf_counter()
+    while True:
+        fn()
+        reps += 1
+        dt = time.perf_counter() - t
+        if dt >= args.cpu_seconds or reps >= 10000:
+            break
     cores = 1 if wl in ("per_token", "swiglu", "swiglu_fp8") else _threads_used()
-    out = {"value": units / dt, "unit": unit, "cores": cores, "kind": "oracle",
-           "sample": desc, "seconds": dt}
+    out = {"value": units * reps / dt, "unit": unit, "cores": cores, "kind": "oracle",
+           "sample": f"{desc}, {reps} run(s)", "seconds": dt}
     if not args.no_all_cores:
         allc = _all_cores(wl)
         if allc is not None:
@@ -685,6 +693,8 @@ def main():
     ap.add_argument("--m", type=int, default=32, help="tokens of the decode workload")
     ap.add_argument("--a-layout", default="128x4", choices=["128x4", "8x4"])
     ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="cpu_baseline repeats its oracle sample until this much time has run")
     ap.add_argument("--no-all-cores", action="store_true",
                     help="skip the oracle timing on all host cores (cpu_baseline.all_cores)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

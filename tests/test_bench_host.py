@@ -56,3 +56,29 @@ def test_decode_f32_and_prefill(bench):
     assert a["read"] == 28672 * 4096 + 28672 * 512 + 32 * 4096 + 32 * 512 * 4
     p = bench.algorithmic("prefill", M=8192, N=8192, K=8192)
     assert p["flops"] == 2 * 8192 ** 3 == 1_099_511_627_776
+
+
+def test_workload_config_shared_by_both_arms(bench):
+    """Both arms print the same workload keys; the GEMM ones carry the shapes they run."""
+    import types
+    args = types.SimpleNamespace(m=32, a_layout="128x4")
+    for wl in ("per_token", "swiglu", "swiglu_fp8"):
+        assert "workload" in bench.workload_config(wl, args)
+    shapes = {"decode": (32, 28672, 8192), "decode_f32": (32, 28672, 8192),
+              "prefill": (8192, 8192, 8192), "tiny": (16, 256, 512)}
+    for wl, mnk in shapes.items():
+        c = bench.workload_config(wl, args)
+        assert (c["M"], c["N"], c["K"]) == mnk
+    assert bench.workload_config("decode_f32", args)["a_scales"] == "fp32 [M, K/16]"
+
+
+def test_cpu_baseline_repeats_the_sample(bench):
+    """The single-thread oracle baseline repeats its bounded sample until the time budget
+    has run and scales the value by the repetitions (the tiny GEMM, a few ms per run)."""
+    import types
+    args = types.SimpleNamespace(cpu_rows=2048, m=32, a_layout="128x4", no_all_cores=True,
+                                 cpu_seconds=0.2)
+    r = bench.cpu_baseline("tiny", args)
+    reps = int(r["sample"].rsplit(", ", 1)[1].split()[0])
+    assert reps >= 1 and r["seconds"] >= 0.2
+    assert r["kind"] == "oracle" and r["unit"] == "TFLOP/s" and r["value"] > 0
