@@ -37,3 +37,22 @@ def test_oracle_includes_no_cuda_path_header():
     ours = {os.path.basename(p) for p in glob.glob(os.path.join(PKG, "csrc", "*"))}
     ours |= {os.path.basename(p) for p in glob.glob(os.path.join(ROOT, "include", "*.h"))}
     assert includes and not (set(map(os.path.basename, includes)) & ours), includes
+
+
+def test_bench_loads_the_oracle_only_for_its_baselines():
+    """bench.py imports the oracle inside its CPU-baseline and reference-arm functions only."""
+    code = ("import sys, importlib.util; sys.path.insert(0, %r)\n"
+            "spec = importlib.util.spec_from_file_location('bench', %r)\n"
+            "m = importlib.util.module_from_spec(spec); spec.loader.exec_module(m)\n"
+            "print('oracle' in sys.modules)") % (ROOT, os.path.join(ROOT, "bench.py"))
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.strip().splitlines()[-1] == "False"
+    with open(os.path.join(ROOT, "bench.py")) as fh:
+        src = fh.read()
+    users = set()
+    for fn in re.finditer(r"^def (\w+)\(.*?(?=^def |\Z)", src, re.M | re.S):
+        if re.search(r"^\s+import oracle\b", fn.group(0), re.M):
+            users.add(fn.group(1))
+    assert users and users <= {"_oracle_sample", "cpu_baseline", "_all_cores", "_oracle_rows",
+                               "run_reference"}, users
