@@ -146,3 +146,37 @@ def test_missing_library_fails_loudly(monkeypatch):
     x = torch.zeros(4, 32, dtype=torch.bfloat16)
     with pytest.raises(RuntimeError, match="not built"):
         nv.nvfp4_quantize(x, torch.ones(1))
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "nvfp4.h"
+
+int main(void) {
+  /* host-only entry points: sizes, status strings and argument checks (no device touched) */
+  long long a = (long long)nvfp4_sf_bytes(200, 96, NVFP4_SF_128x4);  /* 256 rows x 8 columns */
+  long long b = (long long)nvfp4_sf_bytes(9, 64, NVFP4_SF_8x4);      /* 16 rows x 4 columns */
+  int bad = nvfp4_quantize(NULL, NVFP4_IN_BF16, 1, 17, 17, NULL, 0, NULL, NULL, NVFP4_SF_128x4, NULL);
+  printf("%lld %lld %d %s\n", a, b, bad, nvfp4_status_str(bad));
+  return strcmp(nvfp4_status_str(NVFP4_OK), "NVFP4_OK") != 0;
+}
+"""
+
+
+def test_plain_c_client_compiles_links_and_runs(L, tmp_path):
+    """The boundary used from C: the header compiles as pedantic C99 and a program linked
+    against libnvfp4.so gets the documented sizes and argument errors."""
+    import subprocess
+
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(nv.LIB_PATH)
+    cmd = ["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+           str(src), "-o", str(exe), "-L", libdir, "-l:libnvfp4.so", "-Wl,-rpath," + libdir]
+    build = subprocess.run(cmd, capture_output=True, text=True, timeout=120)
+    assert build.returncode == 0, build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert run.returncode == 0, run.stderr
+    assert run.stdout.split() == [str(256 * 8), str(16 * 4), "1", "NVFP4_ERR_INVALID_ARG"]
