@@ -309,3 +309,30 @@ def test_gemm_row_parallel_reading(orc):
         assert np.all(np.abs(got - full64) <= bound)
     with pytest.raises(AssertionError):
         orc.gemm_row_parallel(a[:, :96], sa[:, :12], 2.0, w[:, :96], sw[:, :12], 30.0, tp=2)
+
+
+def test_gemm_row_parallel_rounds_each_rank(orc):
+    """Each rank's output is rounded to fp16 before the AllReduce adds it ("Fused Nvfp4 GEMM
+    All Reduce Plugin": rank-local FP16 [B,N] output, then the AllReduce). A hand-built case
+    where that rounding decides the result, M = N = 1, K = 128, tp = 2, unit global scales:
+      rank 0 (K 0..63):   1*1 (scales 1) + 0.5*0.5 (scales 2^-4, 2^-4)           = 1 + 2^-10
+      rank 1 (K 64..127): 1*1 + 0.5*0.5 (2^-4, 2^-4) + 0.5*0.5 (2^-4, 2^-5)
+                          + 0.5*0.5 (2^-5, 2^-5)                  = 1 + 7*2^-12 -> fp16 1 + 2^-9
+    The fp16 partials add to 2 + 3*2^-10, halfway between fp16 2 + 2^-9 and 2 + 2^-8, which
+    rounds to the even 2 + 2^-8 (0x4002). Adding the unrounded partials instead gives
+    2 + 11*2^-12, which rounds to 2 + 2^-9 (0x4001)."""
+    one, half = 0x2, 0x1                                # E2M1 codes of 1.0 and 0.5
+    s1, s4, s5 = 0x38, 0x18, 0x10                       # E4M3 codes of 1, 2^-4, 2^-5
+    codes_a, codes_w = np.zeros(128, np.uint8), np.zeros(128, np.uint8)
+    sa, sw = np.full((1, 8), s1, np.uint8), np.full((1, 8), s1, np.uint8)
+    for blk, (ca, cw, xa, xw) in {0: (one, one, s1, s1), 1: (half, half, s4, s4),
+                                  4: (one, one, s1, s1), 5: (half, half, s4, s4),
+                                  6: (half, half, s4, s5), 7: (half, half, s5, s5)}.items():
+        codes_a[16 * blk], codes_w[16 * blk] = ca, cw
+        sa[0, blk], sw[0, blk] = xa, xw
+    pack = lambda c: (c[0::2] | (c[1::2] << 4)).astype(np.uint8).reshape(1, 64)  # noqa: E731
+    a, w = pack(codes_a), pack(codes_w)
+    out16, sum64 = orc.gemm_row_parallel(a, sa, 1.0, w, sw, 1.0, tp=2, want_f64=True)
+    assert sum64[0, 0] == 2 + 11 * 2.0 ** -12
+    assert out16[0, 0] == 0x4002
+    assert orc.gemm(a, sa, 1.0, w, sw, 1.0)[0, 0] == 0x4001   # the one-rank GEMM of the same data
