@@ -3,7 +3,11 @@ routine behind "feature: add fp4 mm using trtllm backend" (FlashInfer PR #1355),
 writes both layouts. FlashInfer quantizes the same input three times (linear, 128x4, 8x4
 scales); the oracle's swizzle of FlashInfer's own linear scales must reproduce its swizzled
 bytes exactly, padding included. Only the byte permutation is compared, so the two
-quantizers' arithmetic does not enter. No kernel of this library runs here."""
+quantizers' arithmetic does not enter. No kernel of this library runs here.
+
+FlashInfer is part of the GPU image: if it cannot be imported these tests fail (they are
+the live form of the layout pin; tests/golden/flashinfer_sf_layouts.txt holds FlashInfer's
+bytes for a few ragged shapes so that the pin also holds on the CPU)."""
 import numpy as np
 import pytest
 import torch
@@ -14,10 +18,18 @@ from tests.helpers import require_cuda
 pytestmark = pytest.mark.gpu
 
 
+def _flashinfer():
+    try:
+        import flashinfer
+    except Exception as e:  # a missing library must not turn the pin into a skip
+        pytest.fail(f"flashinfer is needed for the layout pin and could not be imported: {e}")
+    return flashinfer
+
+
 @pytest.mark.parametrize("M,K", [(40, 512), (130, 320), (17, 64), (256, 1024)])
 def test_scale_layouts_match_flashinfer(M, K):
     require_cuda()
-    flashinfer = pytest.importorskip("flashinfer")
+    flashinfer = _flashinfer()
     g = torch.Generator(device="cuda").manual_seed(M * 7 + K)
     # block magnitudes spread over several binades so the scale codes vary
     x = torch.randn(M, K, device="cuda", generator=g) * torch.exp(
@@ -57,7 +69,7 @@ def test_quantize_against_flashinfer(M, K, seed, dtype):
     reciprocals, so a packed value may land one E2M1 step away where x * r sits at a rounding
     midpoint: fewer than 1% of bytes may differ, by one step, with the same sign."""
     require_cuda()
-    flashinfer = pytest.importorskip("flashinfer")
+    flashinfer = _flashinfer()
     from nvfp4_block_scaled_10_b200 import workloads
     x = workloads.per_token(M, K, seed=seed).to(dtype)
     odt = orc.BF16 if dtype == torch.bfloat16 else orc.FP16

@@ -336,3 +336,33 @@ def test_gemm_row_parallel_rounds_each_rank(orc):
     assert sum64[0, 0] == 2 + 11 * 2.0 ** -12
     assert out16[0, 0] == 0x4002
     assert orc.gemm(a, sa, 1.0, w, sw, 1.0)[0, 0] == 0x4001   # the one-rank GEMM of the same data
+
+
+def test_flashinfer_sf_layout_bytes(orc):
+    """The 128x4 and 8x4 layouts pinned to FlashInfer's own bytes on the CPU: for each shape
+    in tests/golden/flashinfer_sf_layouts.txt (written on a GPU by
+    tests/golden/make_flashinfer_sf_layouts.py, which runs only FlashInfer's fp4_quantize,
+    the routine of "feature: add fp4 mm using trtllm backend" that introduced both layouts),
+    the oracle's swizzle of FlashInfer's linear scales must give FlashInfer's 128x4 and 8x4
+    buffers byte for byte, padding included. Shapes have ragged rows and, for K = 96,
+    ragged scale columns."""
+    path = os.path.join(os.path.dirname(__file__), "golden", "flashinfer_sf_layouts.txt")
+    lines = [ln.strip() for ln in open(path) if ln.strip() and not ln.startswith("#")]
+    shapes = 0
+    ragged_cols = False
+    while lines:
+        head, lin_hex, s128_hex, s84_hex = lines[:4]
+        lines = lines[4:]
+        _, M, K = head.split()
+        M, K = int(M), int(K)
+        C = K // 16
+        lin = np.frombuffer(bytes.fromhex(lin_hex), np.uint8).reshape(M, C)
+        assert len(np.unique(lin)) >= 8
+        for hx, layout in ((s128_hex, orc.L128x4), (s84_hex, orc.L8x4)):
+            want = np.frombuffer(bytes.fromhex(hx), np.uint8)
+            got = orc.swizzle(lin, layout)
+            assert got.size == want.size, (M, K, layout, got.size, want.size)
+            assert np.array_equal(got, want), (M, K, layout)
+        shapes += 1
+        ragged_cols |= C % 4 != 0
+    assert shapes >= 2 and ragged_cols

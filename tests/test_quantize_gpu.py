@@ -1,14 +1,16 @@
 """GPU parity of the quantize kernels against the oracle: bit-exact bytes.
 
 Small shapes span several CTAs, ragged tails and every layout; the full per-token and
-SwiGLU workloads are compared in full."""
+SwiGLU workloads are compared in full. Outputs carry canary guard bands (helpers.Guarded)
+that must be untouched after each launch."""
 import numpy as np
 import pytest
 import torch
 
 import oracle as orc
 from nvfp4_block_scaled_10_b200 import workloads
-from tests.helpers import assert_bytes_equal, host_bytes, require_cuda, to_dev_bits
+from tests.helpers import (Guarded, assert_bytes_equal, check_guards, guarded, host_bytes,
+                           require_cuda, to_dev_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,16 +30,19 @@ def _quantize_both(nv, xt, dtype, per_token, layout, K):
     M = xs.shape[0]
     xd = xt.cuda()[:, :K]
     if per_token:
-        g_dev = torch.full((M,), -1.0, dtype=torch.float32, device="cuda")
+        gg = guarded((M,), torch.float32)
         q_o, sf_o, g_o = orc.quantize(bits, odt, per_token=True)
     else:
         g = orc.global_scale(bits, odt)
-        g_dev = torch.tensor([g], dtype=torch.float32, device="cuda")
+        gg = guarded((1,), torch.float32)
+        gg.view(torch.float32).fill_(g)
         q_o, sf_o, g_o = orc.quantize(bits, odt, g=g)
-    sf_dev = torch.full((nv.nvfp4_sf_bytes(M, K, layout),), 0xAA, dtype=torch.uint8, device="cuda")
-    q_dev = torch.full((M, K // 2), 0xAA, dtype=torch.uint8, device="cuda")
+    gsf = Guarded(nv.nvfp4_sf_bytes(M, K, layout))
+    gq = guarded((M, K // 2))
+    g_dev, q_dev, sf_dev = gg.view(torch.float32), gq.view(torch.uint8, (M, K // 2)), gsf.view()
     nv.nvfp4_quantize(xd, g_dev, per_token=per_token, sf_layout=layout, q=q_dev, sf=sf_dev)
     torch.cuda.synchronize()
+    check_guards(q=gq, sf=gsf, g=gg)
     assert_bytes_equal(host_bytes(q_dev), q_o, "q")
     assert_bytes_equal(host_bytes(sf_dev), orc.swizzle(sf_o, layout), "sf")
     if per_token:
@@ -121,8 +126,11 @@ def test_global_scale_parity(M, K, pad, dtype):
     xt = _inputs(M, K, pad, seed=M + K + pad, dtype=dtype)
     bits = workloads.bits16(xt[:, :K].contiguous())
     g_o = orc.global_scale(bits, DT[dtype][1])
-    g = nv.nvfp4_global_scale(xt.cuda()[:, :K])
+    gg = guarded((1,), torch.float32)
+    gws = Guarded(max(nv.nvfp4_global_scale_workspace_bytes(M, K), 16))
+    g = nv.nvfp4_global_scale(xt.cuda()[:, :K], g_out=gg.view(torch.float32), workspace=gws.view())
     torch.cuda.synchronize()
+    check_guards(g=gg, workspace=gws)
     assert g.item() == g_o
 
 
@@ -144,10 +152,13 @@ def test_swiglu_parity_small(M, H, pad, layout, dtype):
     bits = workloads.bits16(xs)
     g = orc.global_scale_from_amax(orc.swiglu_amax(bits, odt))
     q_o, sf_o = orc.swiglu_quantize(bits, g, odt)
-    sf_dev = torch.full((nv.nvfp4_sf_bytes(M, H, layout),), 0xAA, dtype=torch.uint8, device="cuda")
+    gsf = Guarded(nv.nvfp4_sf_bytes(M, H, layout))
+    gq = guarded((M, H // 2))
     q, sf = nv.swiglu_nvfp4_quantize(xt.cuda()[:, :2 * H], torch.tensor([g], device="cuda"),
-                                     sf_layout=layout, sf=sf_dev)
+                                     sf_layout=layout, q=gq.view(torch.uint8, (M, H // 2)),
+                                     sf=gsf.view())
     torch.cuda.synchronize()
+    check_guards(q=gq, sf=gsf)
     assert_bytes_equal(host_bytes(q), q_o, "q")
     assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, layout), "sf")
 
@@ -197,10 +208,12 @@ def test_swizzle_unswizzle_parity(R, C, layout):
     nv = require_cuda()
     lin = workloads.random_bytes((R, C), seed=R + C + layout, low=1, high=255)
     want = orc.swizzle(lin, layout)
-    out = torch.full((want.size,), 0xAA, dtype=torch.uint8, device="cuda")
-    got = nv.nvfp4_sf_swizzle(torch.from_numpy(lin).cuda(), layout, out=out)
-    back = nv.nvfp4_sf_unswizzle(got, R, C, layout)
+    gout = Guarded(want.size)
+    gback = guarded((R, C))
+    got = nv.nvfp4_sf_swizzle(torch.from_numpy(lin).cuda(), layout, out=gout.view())
+    back = nv.nvfp4_sf_unswizzle(got, R, C, layout, out=gback.view(torch.uint8, (R, C)))
     torch.cuda.synchronize()
+    check_guards(swizzled=gout, unswizzled=gback)
     assert_bytes_equal(host_bytes(got), want, "swizzle")
     assert_bytes_equal(host_bytes(back), lin, "unswizzle")
 
@@ -211,10 +224,15 @@ def test_per_token_workload_full():
     """[8192, 7168] bf16 with 0.1% x50 outliers, per-token g, 128x4 scales: every byte."""
     nv = require_cuda()
     x = workloads.per_token()
+    M, K = x.shape
     bits = workloads.bits16(x)
     q_o, sf_o, g_o = orc.quantize(bits, orc.BF16, per_token=True)
-    q, sf, g = nv.nvfp4_quantize(x.cuda(), per_token=True, sf_layout=nv.SF_128x4)
+    gq, gsf, gg = guarded((M, K // 2)), Guarded(nv.nvfp4_sf_bytes(M, K, nv.SF_128x4)), guarded((M,), torch.float32)
+    q, sf, g = nv.nvfp4_quantize(x.cuda(), gg.view(torch.float32), per_token=True,
+                                 sf_layout=nv.SF_128x4, q=gq.view(torch.uint8, (M, K // 2)),
+                                 sf=gsf.view())
     torch.cuda.synchronize()
+    check_guards(q=gq, sf=gsf, g=gg)
     assert_bytes_equal(host_bytes(g), g_o.view(np.uint8), "g")
     assert_bytes_equal(host_bytes(q), q_o, "q")
     assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, orc.L128x4), "sf")
@@ -224,12 +242,16 @@ def test_swiglu_workload_full():
     """[4096, 2 x 14336] bf16, per-tensor g from amax(Y) by the oracle, 128x4: every byte."""
     nv = require_cuda()
     x = workloads.swiglu()
+    M, H = x.shape[0], x.shape[1] // 2
     bits = workloads.bits16(x)
     g = orc.global_scale_from_amax(orc.swiglu_amax(bits, orc.BF16))
     q_o, sf_o = orc.swiglu_quantize(bits, g, orc.BF16)
+    gq, gsf = guarded((M, H // 2)), Guarded(nv.nvfp4_sf_bytes(M, H, nv.SF_128x4))
     q, sf = nv.swiglu_nvfp4_quantize(x.cuda(), torch.tensor([g], device="cuda"),
-                                     sf_layout=nv.SF_128x4)
+                                     sf_layout=nv.SF_128x4, q=gq.view(torch.uint8, (M, H // 2)),
+                                     sf=gsf.view())
     torch.cuda.synchronize()
+    check_guards(q=gq, sf=gsf)
     assert_bytes_equal(host_bytes(q), q_o, "q")
     assert_bytes_equal(host_bytes(sf), orc.swizzle(sf_o, orc.L128x4), "sf")
 
@@ -264,8 +286,11 @@ def test_swiglu_fp8_parity(M, H, pad, scale, dtype):
     x = workloads.normal((M, 2 * H + pad), 1.0, seed=M + H, dtype=tdt)
     xs = x[:, :2 * H].contiguous()
     q_o = orc.swiglu_fp8(workloads.bits16(xs), scale, odt)
-    q = nv.swiglu_fp8_quantize(x.cuda()[:, :2 * H], torch.tensor([scale], device="cuda"))
+    gq = guarded((M, H))
+    q = nv.swiglu_fp8_quantize(x.cuda()[:, :2 * H], torch.tensor([scale], device="cuda"),
+                               q=gq.view(torch.uint8, (M, H)))
     torch.cuda.synchronize()
+    check_guards(q=gq)
     assert_bytes_equal(host_bytes(q), q_o, "q")
 
 
@@ -292,6 +317,9 @@ def test_swiglu_fp8_workload_full():
     x = workloads.swiglu(4096, 14336)
     scale = 448.0 / 60.0
     q_o = orc.swiglu_fp8(workloads.bits16(x), scale, orc.BF16)
-    q = nv.swiglu_fp8_quantize(x.cuda(), torch.tensor([scale], device="cuda"))
+    gq = guarded((4096, 14336))
+    q = nv.swiglu_fp8_quantize(x.cuda(), torch.tensor([scale], device="cuda"),
+                               q=gq.view(torch.uint8, (4096, 14336)))
     torch.cuda.synchronize()
+    check_guards(q=gq)
     assert_bytes_equal(host_bytes(q), q_o, "q")

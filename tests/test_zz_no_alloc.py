@@ -4,9 +4,9 @@ plan that forbids per-call cudaMalloc/cudaFree). Its reduction scratch is a stat
 inside the library, so the call takes no workspace.
 
 The GPU test calls the new entry point through the C ABI and checks it against the
-workspace-taking nvfp4_global_scale (bit-identical g, the tolerance every global-scale test
-here uses) on consecutive calls, the second smaller than the first so stale partials from
-the first call would show. This file sorts last so a stop-at-first-failure run has already
+workspace-taking nvfp4_global_scale and against the oracle's global scale (bit-identical g,
+the tolerance every global-scale test here uses) on consecutive calls, the second smaller
+than the first so stale partials from the first call would show. This file sorts last so a stop-at-first-failure run has already
 run everything else."""
 import ctypes
 
@@ -14,6 +14,7 @@ import pytest
 import torch
 
 import nvfp4_block_scaled_10_b200 as nv
+import oracle as orc
 from nvfp4_block_scaled_10_b200 import workloads
 
 
@@ -61,4 +62,6 @@ def test_noalloc_matches_workspace_entry_point_on_consecutive_calls():
         assert L.nvfp4_global_scale_noalloc(_c(x), dtype, M, K, K, _c(g_new), stream) == nv.OK
         torch.cuda.synchronize()
         assert g_new.item() == g_ref.item(), (M, K, g_new.item(), g_ref.item())
+        g_orc = orc.global_scale(workloads.bits16(x_host), orc.BF16 if dtype == 0 else orc.FP16)
+        assert g_new.item() == g_orc, (M, K, g_new.item(), g_orc)
         assert g_new.item() > 0
