@@ -152,9 +152,9 @@ NVFP4_API int nvfp4_quantize(const void *x, int dtype, int64_t M, int64_t K, int
  * Kernel in CUDA": the activation is computed in fp32 registers and only the quantized
  * result is written; here the output is NVFP4 instead of FP8).
  *   y[m,h] = silu(x[m,h]) * x[m,H+h],  silu(v) = v / (1 + e(-v)),
- * where e() is the library's fp32 exponential (clamp to [-87, 88], k = rint(v*log2 e),
- * Cody-Waite reduction with ln2 = 0x3F317200 + 0x35BFBE8E, degree-7 Taylor polynomial by
- * fused multiply-add, times 2^k). y stays fp32 and is quantized exactly as in
+ * where e() is the library's fp32 exponential (clamp to [-87, 88]; k = the integer nearest
+ * the exact product v * fl(log2 e), ties to even; Cody-Waite reduction with ln2 =
+ * 0x3F317200 + 0x35BFBE8E; degree-7 Taylor polynomial by fused multiply-add; times 2^k). y stays fp32 and is quantized exactly as in
  * nvfp4_quantize with the per-tensor scale g[0]. Y is never written to memory.
  * x   device, [M, 2H] `dtype` (gate = columns [0,H), up = columns [H,2H)), row stride ldx.
  * g   device, one fp32, read.
@@ -227,8 +227,11 @@ NVFP4_API size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  *          nvfp4_gemm_workspace_bytes).
  * dev_status: device int32 or NULL. Each bounded wait inside the kernel that gives up
  *          (about 2 s without progress) ORs 1 into it and the kernel returns without
- *          finishing; a split-K tile counter found non-zero on entry (a workspace that was
- *          not zero-filled) ORs 4. The caller reads it after synchronizing.
+ *          finishing. A split-K tile counter found at or above its tile's piece count (a
+ *          workspace that was not zero-filled) ORs 4. A counter left part-way by a call
+ *          that gave up is NOT detected by the next call, which would then add stale
+ *          partial sums: after any call that set a dev_status bit, zero-fill the workspace
+ *          again before reusing it. The caller reads dev_status after synchronizing.
  * Requires: K % 64 == 0, N % 8 == 0, a_q/w_q/a_sf/w_sf/out 16-byte aligned, a_layout in
  *          {128x4, 8x4} (8x4 only when M <= 32).
  */
@@ -277,8 +280,9 @@ NVFP4_API int nvfp4_gemm_per_token(const uint8_t *a_q, const uint8_t *a_sf, int 
  *          (M, N, K); used as in nvfp4_gemm, plus the plane words (K/64 x 384 bytes) and 32
  *          row factors of one 32-row chunk after the partial tiles, rewritten by every call.
  * dev_status: device int32 or NULL; bit 1 a bounded wait gave up (NVFP4_ERR_TIMEOUT), bit 2
- *          a bad activation scale, bit 4 a workspace that was not zero-filled. The caller
- *          reads it after synchronizing.
+ *          a bad activation scale, bit 4 a workspace that was not zero-filled (detected as
+ *          in nvfp4_gemm: zero-fill the workspace again after any call that set a bit). The
+ *          caller reads it after synchronizing.
  * Requires: K % 64 == 0, N % 8 == 0.
  */
 NVFP4_API size_t nvfp4_gemm_act_f32_workspace_bytes(int64_t M, int64_t N, int64_t K);

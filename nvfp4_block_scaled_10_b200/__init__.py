@@ -46,6 +46,12 @@ SIGNATURES = {
                                   _vp]),
 }
 
+# test hooks declared in include/nvfp4_testing.h (they change no result; see that header)
+TESTING_SIGNATURES = {
+    "nvfp4_testing_set_wait_limit": (_i32, [ctypes.c_uint64]),
+    "nvfp4_testing_withhold_stage": (_i32, [_i32, _i64]),
+}
+
 _lib = None
 
 
@@ -63,7 +69,7 @@ def lib() -> ctypes.CDLL:
             raise RuntimeError(f"libnvfp4.so is not built ({LIB_PATH}); run "
                                "`python -m nvfp4_block_scaled_10_b200.build`")
         L = ctypes.CDLL(LIB_PATH)
-        for name, (res, args) in SIGNATURES.items():
+        for name, (res, args) in {**SIGNATURES, **TESTING_SIGNATURES}.items():
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args

@@ -541,6 +541,9 @@ struct DecParams {
   int tile_base;        // = grid x full_per_cta; tiles from here on are split stream-K
   int64_t rem_units;    // (tiles - tile_base) x K-steps, cut evenly over CTAs 0 .. rem_ctas - 1
   int rem_ctas;         // min(grid, rem_units): every one of them gets at least one unit
+  uint64_t wait_ns;     // limit of every bounded wait (2 s unless a test hook shortens it)
+  int withhold_cta;     // test hook: CTA whose producer stops at ring position withhold_it
+  int withhold_it;      // (-1: none; E4M3 activation scales only)
 };
 
 // Contiguous unit range [u0, u1) of CTA c among G over U units (units = tile x K-step).
@@ -713,8 +716,14 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       for (int kt = kb; kt < ke; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
+        // test hook: this CTA issues nothing from this ring position on, so its consumers'
+        // bounded waits run out with no copy in flight
+        if (NPL == 1 && c == p.withhold_cta && static_cast<int>(it) == p.withhold_it) {
+          ok = false;
+          break;
+        }
         if (!planes_out && it == STAGES) issue_first_planes(STAGES);
-        if (it >= STAGES && !mbar_wait_warp(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
+        if (it >= STAGES && !mbar_wait_warp(&empty[stage], (round - 1) & 1, p.wait_ns)) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
           break;
@@ -752,7 +761,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       const uint32_t used = it < STAGES ? it : STAGES;
       for (uint32_t i = 0; i < used; ++i) {
         const uint32_t j = it - used + i;
-        if (!mbar_wait_warp(&empty[j % STAGES], (j / STAGES) & 1, kWaitTimeoutNs)) {
+        if (!mbar_wait_warp(&empty[j % STAGES], (j / STAGES) & 1, p.wait_ns)) {
           if (lane == 0) report_timeout(p.dev_status);
           break;
         }
@@ -768,18 +777,19 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       for (; ok && itr.next(tile, kb, ke); ++seg) {
         const int buf = static_cast<int>(seg % C::kAccBufs);
         const uint32_t use = seg / C::kAccBufs;
-        if (use > 0 && !mbar_wait_bounded(&acc_empty[buf], (use - 1) & 1, kWaitTimeoutNs)) {
+        if (use > 0 && !mbar_wait_bounded(&acc_empty[buf], (use - 1) & 1, p.wait_ns)) {
           report_timeout(p.dev_status);
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + buf * C::kAccCols;
         int prev = -1;
+        uint32_t prev_round = 0;
         for (int kt = kb; kt < ke; ++kt, ++it) {
           const int stage = static_cast<int>(it % STAGES);
           const uint32_t round = it / STAGES;
-          if (!mbar_wait_bounded(&full[stage], round & 1, kWaitTimeoutNs) ||
-              !mbar_wait_bounded(&sf_full[stage], round & 1, kWaitTimeoutNs)) {
+          if (!mbar_wait_bounded(&full[stage], round & 1, p.wait_ns) ||
+              !mbar_wait_bounded(&sf_full[stage], round & 1, p.wait_ns)) {
             report_timeout(p.dev_status);
             ok = false;
             break;
@@ -795,9 +805,14 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
                      slot + kK64PerStage * 4 + a * 4, (kt != kb || a != 0) ? 1u : 0u);
           }
           prev = stage;
+          prev_round = round;
         }
         if (prev >= 0) tc_commit(&empty[prev]);
         if (ok) tc_commit(&acc_full[buf]);
+        // after a timeout the producer skips its final waits on the stages' releases, so the
+        // MMAs issued so far are waited for here: none is in flight when the CTA frees its
+        // tensor memory
+        if (!ok && prev >= 0) (void)mbar_wait_bounded(&empty[prev], prev_round & 1, p.wait_ns);
       }
     }
     __syncwarp();
@@ -807,7 +822,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     uint32_t it = 0;
     bool ok = true;
-    if (p.a_sf_8x4 && !mbar_wait_warp(sfb_ready, 0, kWaitTimeoutNs)) {
+    if (p.a_sf_8x4 && !mbar_wait_warp(sfb_ready, 0, p.wait_ns)) {
       if (lane == 0) report_timeout(p.dev_status);
       ok = false;
     }
@@ -821,7 +836,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         const uint32_t round = it / STAGES;
         const int k64_0 = kt * kK64PerStage;
         const int nk64 = min(kK64PerStage, num_k64 - k64_0);
-        if (!mbar_wait_warp(&full[stage], round & 1, kWaitTimeoutNs)) {
+        if (!mbar_wait_warp(&full[stage], round & 1, p.wait_ns)) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
           break;
@@ -875,7 +890,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       const int buf = static_cast<int>(seg % C::kAccBufs);
       const uint32_t use = seg / C::kAccBufs;
       // the four epilogue warps leave together (they meet at named barriers below)
-      const bool got = mbar_wait_warp(&acc_full[buf], use & 1, kWaitTimeoutNs);
+      const bool got = mbar_wait_warp(&acc_full[buf], use & 1, p.wait_ns);
       if (!epi_all(got, C::kEpiWarps * 32)) {
         if (lane == 0) report_timeout(p.dev_status);
         break;
@@ -932,7 +947,9 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
         const int old = atomicAdd(p.counters + st, 1);
         *last_flag = (old == pieces - 1) ? 1 : 0;
         // the last arriver hands the counter back zeroed for the next call on this
-        // workspace; a count past the pieces means the workspace was not zero on entry
+        // workspace; a count past the pieces means the workspace was not zero on entry (a
+        // count left part-way by a call that gave up cannot be told from a live one, so the
+        // caller zero-fills the workspace again after any dev_status error)
         if (old == pieces - 1) atomicExch(p.counters + st, 0);
         if ((old < 0 || old >= pieces) && p.dev_status != nullptr) atomicOr(p.dev_status, kDevErrWorkspace);
       }
@@ -1597,6 +1614,10 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(g.workspace) +
                                          counter_region(g.workspace_bytes));
   p.dev_status = g.dev_status;
+  const DebugHooks hooks = debug_hooks();
+  p.wait_ns = hooks.wait_ns;
+  p.withhold_cta = hooks.withhold_cta;
+  p.withhold_it = static_cast<int>(hooks.withhold_it);
   cudaError_t e = cudaSuccess;
   const int smem = C::smem_bytes(static_cast<int>(g.K / 64), p.a_sf_8x4 != 0);
   e = ensure_smem_attr(gemm_nvfp4_decode_kernel<STAGES, NPL>, smem);

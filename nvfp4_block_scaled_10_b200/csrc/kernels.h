@@ -18,6 +18,14 @@ constexpr int kDevErrTimeout = 1;
 constexpr int kDevErrBadScale = 2;  // an fp32 activation scale was negative, NaN or infinite
 constexpr int kDevErrWorkspace = 4;  // a split-K tile counter was not zero when the call began
 
+// testing.cu: the hooks of include/nvfp4_testing.h as the launchers read them.
+struct DebugHooks {
+  uint64_t wait_ns;      // limit of the small-M GEMM's bounded waits
+  int withhold_cta;      // CTA whose producer stops at ring position withhold_it (-1: none)
+  int64_t withhold_it;
+};
+DebugHooks debug_hooks();
+
 // quantize.cu
 int *device_error_symbol();
 int global_scale_parts(int64_t M, int64_t K, int num_sms);

@@ -3,9 +3,10 @@
 //  * global amax -> per-tensor encode scale g (two launches, partial maxima in workspace)
 //  * streaming quantize: one thread owns one 16-element block (one 32-byte load), given g
 //    per tensor or per row
-//  * per-token quantize: whole rows staged in shared memory by bulk TMA copies (several rows
-//    in flight per CTA), row amax -> g_row, then the blocks of the row are quantized from
-//    shared memory, so X is read from HBM once
+//  * per-token quantize: one row per CTA at a time held in registers (the next row streams
+//    into the registers as they free), row amax -> g_row, then the blocks of the row are
+//    quantized from the same registers, so X is read from HBM once (rows longer than
+//    32768 elements take a two-pass path that reads X twice)
 //  * fused SwiGLU + quantize: y = silu(gate) * up formed in registers, never stored
 //  * scale-layout swizzle / unswizzle
 //

@@ -13,8 +13,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "nvfp4.h")
 
 
-def _declared_symbols():
-    text = open(HEADER).read()
+TESTING_HEADER = os.path.join(ROOT, "include", "nvfp4_testing.h")
+
+
+def _declared_symbols(header=HEADER):
+    text = open(header).read()
     return sorted(set(re.findall(r"^NVFP4_API\s+[\w\s\*]*?\b(\w+)\s*\(", text, re.M)))
 
 
@@ -32,9 +35,17 @@ def test_header_declares_the_boundary():
 
 
 def test_library_exports_every_declared_symbol(L):
-    for name in _declared_symbols():
+    for name in _declared_symbols() + _declared_symbols(TESTING_HEADER):
         assert hasattr(L, name), name
         assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_testing_header_declares_the_hooks(L):
+    assert _declared_symbols(TESTING_HEADER) == sorted(nv.TESTING_SIGNATURES)
+    # host-only setters: defaults restored, out-of-range positions refused
+    assert L.nvfp4_testing_set_wait_limit(0) == nv.OK
+    assert L.nvfp4_testing_withhold_stage(-1, -1) == nv.OK
+    assert L.nvfp4_testing_withhold_stage(0, 1 << 40) == nv.ERR_INVALID_ARG
 
 
 def test_status_strings(L):
