@@ -379,6 +379,82 @@ __global__ void __launch_bounds__(NT, MINB) quant_pertoken_regs_kernel(
 
 // ------------------------------------------------------------------------------ SwiGLU
 
+// SiLU table for bfloat16 gates. silu(gate) depends on the 16-bit gate alone, so each CTA of
+// the fused SwiGLU kernels first evaluates it once for every bf16 gate with 2^-26 <= |gate| <
+// 2^7 (biased exponents 101..133, both signs: 8448 values, 33 KB of shared memory) with the
+// same arithmetic as the per-element path (silu_pair_neg, whose forms agree bit for bit on
+// every gate), and then looks silu up instead of evaluating the exponential and the division
+// per element. A block takes the table path when all 16 gates are numbers inside that range
+// (a NaN-propagating packed maximum and a packed minimum of |gate| decide it); any other block
+// (zeros, tiny, huge, infinite or NaN gates) evaluates silu per element as before.
+constexpr uint32_t kSiluTabLo = 0x3280u;  // bf16 magnitude bits of 2^-26
+constexpr uint32_t kSiluTabHi = 0x4300u;  // bf16 magnitude bits of 2^7 (first value past the table)
+constexpr uint32_t kSiluTabHalf = kSiluTabHi - kSiluTabLo;  // 4224 entries per sign
+constexpr int kSiluTabEntries = 2 * kSiluTabHalf;            // positive gates, then negative
+constexpr int kSiluTabBytes = kSiluTabEntries * 4;
+
+// Fills the table (all threads of the CTA; the caller synchronises before any lookup).
+__device__ __forceinline__ void build_silu_table(float *tab) {
+  for (int j = 2 * static_cast<int>(threadIdx.x); j < kSiluTabEntries; j += 2 * blockDim.x) {
+    // entries j and j + 1 hold the same sign (kSiluTabHalf is even)
+    const uint32_t mag = kSiluTabLo + static_cast<uint32_t>(j) % kSiluTabHalf;
+    const uint32_t sign = j < static_cast<int>(kSiluTabHalf) ? 0u : 0x80000000u;
+    // silu_pair_neg takes -gate; a bf16 pattern is the upper half of its fp32 value
+    const F2 v{__uint_as_float((mag << 16) ^ sign ^ 0x80000000u),
+               __uint_as_float(((mag + 1u) << 16) ^ sign ^ 0x80000000u)};
+    const F2 sv = silu_pair_neg<true, false>(v);
+    tab[j] = sv.x;
+    tab[j + 1] = sv.y;
+  }
+}
+
+// True when every one of the 16 bf16 gates of a block is a number with 2^-26 <= |gate| < 2^7.
+__device__ __forceinline__ bool silu_table_covers(const uint32_t (&w)[8]) {
+  uint32_t hi0 = w[0], hi1 = w[1], lo0 = w[0], lo1 = w[1];
+#pragma unroll
+  for (int i = 2; i < 8; i += 2) {
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(hi0) : "r"(w[i]));
+    asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(hi1) : "r"(w[i + 1]));
+    asm("min.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(lo0) : "r"(w[i]));
+    asm("min.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(lo1) : "r"(w[i + 1]));
+  }
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(hi0) : "r"(hi1));
+  asm("min.xorsign.abs.bf16x2 %0, %0, %1;" : "+r"(lo0) : "r"(lo1));
+  // clear the signs xorsign left; a NaN magnitude compares above kSiluTabHi too
+  const uint32_t hmax = hi0 & 0x7FFF7FFFu, hmin = lo0 & 0x7FFF7FFFu;
+  return max(hmax & 0xFFFFu, hmax >> 16) < kSiluTabHi && min(hmin & 0xFFFFu, hmin >> 16) >= kSiluTabLo;
+}
+
+__device__ __forceinline__ float lds_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+
+// y = silu(gate) * up for one block from the table (silu_table_covers(wg) must hold; tab is
+// the table's shared-memory address). Returns max |y|. For a packed pair of gates the two
+// table indices come out of one 32-bit computation with 16-bit lanes: idx = magnitude -
+// kSiluTabLo, plus kSiluTabHalf for a negative gate, i.e. bits - kSiluTabLo - sign * (0x8000 -
+// kSiluTabHalf); no lane borrows from or carries into the other for gates in the table.
+__device__ __forceinline__ float swiglu_block16_tab(const uint32_t (&wg)[8], const uint32_t (&wu)[8],
+                                                    uint32_t tab, float (&y)[16]) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t s2 = (wg[i] >> 15) & 0x00010001u;
+    const uint32_t idx2 = wg[i] - (kSiluTabLo | (kSiluTabLo << 16)) - s2 * (0x8000u - kSiluTabHalf);
+    const uint32_t off2 = idx2 << 2;  // byte offsets, each below 2^16
+    const F2 sv{lds_f32(tab + (off2 & 0xFFFFu)), lds_f32(tab + (off2 >> 16))};
+    F2 up;
+    unpack2<0>(wu[i], up.x, up.y);
+    const F2 v = mul2f_rn(sv, up);
+    y[2 * i] = v.x;
+    y[2 * i + 1] = v.y;
+    amax = fmaxf(amax, fmaxf(fabsf(v.x), fabsf(v.y)));
+  }
+  return amax;
+}
+
 // y = silu(gate) * up for the 16 elements of one block (8 packed words of each half);
 // returns max |y|.
 template <int DTYPE, bool CLAMP, bool SAFE>
@@ -425,6 +501,7 @@ __global__ void __launch_bounds__(NT, MINB) swiglu_quant_kernel(
     uint8_t *__restrict__ q, uint8_t *__restrict__ sf, int layout, int64_t Rp, int64_t Cp,
     int chunks_per_row) {
   __shared__ float rtab[128];
+  extern __shared__ float silu_tab[];  // bf16 input: the SiLU table (kSiluTabBytes)
   const int C = static_cast<int>(H / 16);
   const float g0 = g[0];
   // item = blockIdx.x + k * gridDim.x as (row r, chunk ch), advanced without a division
@@ -435,6 +512,8 @@ __global__ void __launch_bounds__(NT, MINB) swiglu_quant_kernel(
   uint32_t wg[UNROLL][8], wu[UNROLL][8];
   if (r < M) load_swiglu_item<DTYPE, UNROLL, V8>(x, ldx, H, C, r, ch * (NT * UNROLL) + threadIdx.x, NT, wg, wu);
   fill_recip_table(rtab, g0);
+  if constexpr (DTYPE == 0) build_silu_table(silu_tab);  // while the first item's loads fly
+  const uint32_t tab = smem_u32(silu_tab);
   __syncthreads();
   while (r < M) {
     int64_t rn = r + step_r;
@@ -454,12 +533,16 @@ __global__ void __launch_bounds__(NT, MINB) swiglu_quant_kernel(
       float y[16];
       float amax = 0.0f;
       if (c < C) {
-        // the packed maximum skips NaN: it exceeds 87 only for a gate beyond the exp clamp
-        // and is infinite only for an infinite gate
-        const float gmax = amax16_packed<DTYPE>(wg[u]);
-        if (gmax <= 87.0f) amax = swiglu_block16<DTYPE, false, false>(wg[u], wu[u], y);
-        else if (gmax != INFINITY) amax = swiglu_block16<DTYPE, true, false>(wg[u], wu[u], y);
-        else amax = swiglu_block16<DTYPE, true, true>(wg[u], wu[u], y);
+        if (DTYPE == 0 && silu_table_covers(wg[u])) {
+          amax = swiglu_block16_tab(wg[u], wu[u], tab, y);
+        } else {
+          // the packed maximum skips NaN: it exceeds 87 only for a gate beyond the exp clamp
+          // and is infinite only for an infinite gate
+          const float gmax = amax16_packed<DTYPE>(wg[u]);
+          if (gmax <= 87.0f) amax = swiglu_block16<DTYPE, false, false>(wg[u], wu[u], y);
+          else if (gmax != INFINITY) amax = swiglu_block16<DTYPE, true, false>(wg[u], wu[u], y);
+          else amax = swiglu_block16<DTYPE, true, true>(wg[u], wu[u], y);
+        }
       }
       const int cn = c0n + u * NT;
       if (rn < M && cn < C) {
@@ -487,6 +570,7 @@ template <int DTYPE, int UNROLL, bool V8, int NT, int MINB>
 __global__ void __launch_bounds__(NT, MINB) swiglu_fp8_kernel(
     const uint16_t *__restrict__ x, int64_t M, int64_t H, int64_t ldx,
     const float *__restrict__ scale, uint8_t *__restrict__ q, int chunks_per_row) {
+  extern __shared__ float silu_tab[];  // bf16 input: the SiLU table (kSiluTabBytes)
   const int C = static_cast<int>(H / 16);
   const float sc = scale[0];
   const int64_t step_r = gridDim.x / chunks_per_row;
@@ -495,6 +579,11 @@ __global__ void __launch_bounds__(NT, MINB) swiglu_fp8_kernel(
   int ch = static_cast<int>(blockIdx.x % chunks_per_row);
   uint32_t wg[UNROLL][8], wu[UNROLL][8];
   if (r < M) load_swiglu_item<DTYPE, UNROLL, V8>(x, ldx, H, C, r, ch * (NT * UNROLL) + threadIdx.x, NT, wg, wu);
+  if constexpr (DTYPE == 0) {
+    build_silu_table(silu_tab);  // while the first item's loads fly
+    __syncthreads();
+  }
+  const uint32_t tab = smem_u32(silu_tab);
   while (r < M) {
     int64_t rn = r + step_r;
     int chn = ch + step_ch;
@@ -511,10 +600,14 @@ __global__ void __launch_bounds__(NT, MINB) swiglu_fp8_kernel(
       const int c = c0 + u * NT;
       float y[16];
       if (c < C) {
-        const float gmax = amax16_packed<DTYPE>(wg[u]);
-        if (gmax <= 87.0f) swiglu_block16<DTYPE, false, false>(wg[u], wu[u], y);
-        else if (gmax != INFINITY) swiglu_block16<DTYPE, true, false>(wg[u], wu[u], y);
-        else swiglu_block16<DTYPE, true, true>(wg[u], wu[u], y);
+        if (DTYPE == 0 && silu_table_covers(wg[u])) {
+          swiglu_block16_tab(wg[u], wu[u], tab, y);
+        } else {
+          const float gmax = amax16_packed<DTYPE>(wg[u]);
+          if (gmax <= 87.0f) swiglu_block16<DTYPE, false, false>(wg[u], wu[u], y);
+          else if (gmax != INFINITY) swiglu_block16<DTYPE, true, false>(wg[u], wu[u], y);
+          else swiglu_block16<DTYPE, true, true>(wg[u], wu[u], y);
+        }
       }
       const int cn = c0n + u * NT;
       if (rn < M && cn < C) {
@@ -696,10 +789,11 @@ cudaError_t launch_swiglu_quantize(const void *x, int dtype, int64_t M, int64_t 
   if (grid > M * cpr) grid = M * cpr;
   if (grid < 1) grid = 1;
   const bool v8 = blocks_32b_aligned(x, ldx);
+  const int smem = dtype == kInBf16 ? kSiluTabBytes : 0;
   NVFP4_DISPATCH_DT_V8(dtype, v8,
                        (swiglu_quant_kernel<DT, kUnroll, VV, kNT, kMinB>
-                        <<<static_cast<int>(grid), kNT, 0, st>>>(xp, M, H, ldx, g, q, sf, layout,
-                                                                 Rp, Cp, cpr)));
+                        <<<static_cast<int>(grid), kNT, smem, st>>>(xp, M, H, ldx, g, q, sf, layout,
+                                                                    Rp, Cp, cpr)));
   return cudaGetLastError();
 }
 
@@ -713,9 +807,10 @@ cudaError_t launch_swiglu_fp8(const void *x, int dtype, int64_t M, int64_t H, in
   if (grid > M * cpr) grid = M * cpr;
   if (grid < 1) grid = 1;
   const bool v8 = blocks_32b_aligned(x, ldx);
+  const int smem = dtype == kInBf16 ? kSiluTabBytes : 0;
   NVFP4_DISPATCH_DT_V8(dtype, v8,
                        (swiglu_fp8_kernel<DT, kUnroll, VV, kNT, kMinB>
-                        <<<static_cast<int>(grid), kNT, 0, st>>>(xp, M, H, ldx, scale, q, cpr)));
+                        <<<static_cast<int>(grid), kNT, smem, st>>>(xp, M, H, ldx, scale, q, cpr)));
   return cudaGetLastError();
 }
 

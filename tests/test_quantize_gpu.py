@@ -323,3 +323,33 @@ def test_swiglu_fp8_workload_full():
     torch.cuda.synchronize()
     check_guards(q=gq)
     assert_bytes_equal(host_bytes(q), q_o, "q")
+
+
+@pytest.mark.parametrize("up_value", [1.0, 3.0])
+def test_swiglu_every_bf16_gate(up_value):
+    """Every one of the 65536 bf16 gate patterns (in order, 16 consecutive patterns per block,
+    so each block lies inside or outside the kernels' SiLU table range as a whole, and the
+    blocks around 2^-26 and 2^7 and the zero, subnormal, infinite and NaN patterns take the
+    per-element path) through both fused SwiGLU kernels, bit-exact against the oracle. The
+    FP8 output (scale 1) keeps about four significant bits of each silu(gate) * up, so a
+    table entry taken for a neighbouring gate shows up here."""
+    nv = require_cuda()
+    gates = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(64, 1024)
+    up = np.full((64, 1024), np.float32(up_value)).view(np.uint32) >> 16
+    bits = np.concatenate([gates, up.astype(np.uint16)], axis=1)
+    x = to_dev_bits(bits, torch.bfloat16)
+    # the NVFP4 encoding has no NaN; NaN gates (covered by the FP8 output below) become zeros
+    nan = ((gates & 0x7F80) == 0x7F80) & ((gates & 0x7F) != 0)
+    bits_nv = np.concatenate([np.where(nan, 0, gates).astype(np.uint16), up.astype(np.uint16)], axis=1)
+    x_nv = to_dev_bits(bits_nv, torch.bfloat16)
+    for g in [1.0, 448.0 * 6.0 / 128.0]:
+        q_o, sf_o = orc.swiglu_quantize(bits_nv, g, orc.BF16)
+        q, sf = nv.swiglu_nvfp4_quantize(x_nv, torch.tensor([g], device="cuda"), sf_layout=nv.SF_LINEAR)
+        torch.cuda.synchronize()
+        assert_bytes_equal(host_bytes(q), q_o, f"swiglu nvfp4 q g={g}")
+        assert_bytes_equal(host_bytes(sf), sf_o, f"swiglu nvfp4 sf g={g}")
+    for scale in [1.0, 0.5]:
+        f_o = orc.swiglu_fp8(bits, scale, orc.BF16)
+        f = nv.swiglu_fp8_quantize(x, torch.tensor([scale], device="cuda"))
+        torch.cuda.synchronize()
+        assert_bytes_equal(host_bytes(f), f_o, f"swiglu fp8 scale={scale}")
