@@ -123,6 +123,19 @@ __device__ __forceinline__ void tmem_st_x8(uint32_t taddr, uint4 a, uint4 b) {
                : "memory");
 }
 
+// 32 consecutive TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_st_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, "
+      "%31, %32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -1007,10 +1020,10 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
 //
 // Synchronisation (barriers named by the CTA holding them):
 //   full[s]      even CTA; both producers arrive.expect_tx and both CTAs' tile copies
-//                complete on it (count 2)
+//                complete on it, and the four scale warps of both CTAs arrive once they
+//                wrote their tensor memory (count 2 + 8): the MMA thread waits on one
+//                barrier per stage
 //   sf_ready[s]  each CTA; its own scale atoms landed (count 1, bulk copies)
-//   sf_full[s]   even CTA; the four scale warps of both CTAs wrote their tensor memory
-//                (count 8)
 //   empty[s]     each CTA; pair-MMA commit multicast to both CTAs
 //   acc_full     each CTA; pair-MMA commit multicast after a tile's last MMA
 //   acc_empty    even CTA; the epilogue warps of both CTAs drained the accumulator (count 16)
@@ -1033,8 +1046,8 @@ struct PairCfg {
   static constexpr int kOutBoxBytes = kHalf * 128;
   static constexpr int kOffOut = kOffSfb + STAGES * kSfbBytes;
   static constexpr int kOffBar = kOffOut + 4 * kOutBoxBytes;
-  // full[S], sf_ready[S], sf_full[S], empty[S], acc_full, acc_empty, tmem slot
-  static constexpr int kBarBytes = (4 * STAGES + 2) * 8 + 16;
+  // full[S], sf_ready[S], empty[S], acc_full, acc_empty, tmem slot
+  static constexpr int kBarBytes = (3 * STAGES + 2) * 8 + 16;
   static constexpr int kSmemBytes = kOffBar + kBarBytes + 1024;
   static constexpr int kAccCols = kN;
   static constexpr int kSfaColsPerK64 = 4;
@@ -1063,8 +1076,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
   uint64_t *sf_ready = full + STAGES;
-  uint64_t *sf_full = sf_ready + STAGES;
-  uint64_t *empty = sf_full + STAGES;
+  uint64_t *empty = sf_ready + STAGES;
   uint64_t *acc_full = empty + STAGES;
   uint64_t *acc_empty = acc_full + 1;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 1);
@@ -1083,9 +1095,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 2);
+      mbar_init(&full[s], 2 + 8);  // two producers (with their bytes), eight scale warps
       mbar_init(&sf_ready[s], 1);
-      mbar_init(&sf_full[s], 8);
       mbar_init(&empty[s], 1);
     }
     mbar_init(acc_full, 1);
@@ -1181,18 +1192,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
           break;
         }
         tc_fence_after();
-        int prev = -1;  // stage whose release is still to be issued (see the single-CTA kernel)
+        // One barrier per stage (operands and scales), and the stage is released right after
+        // its MMAs. (Measured on B200 against the single-CTA kernel's order, where a stage is
+        // released only after the next stage's barriers: 2.5 % faster here together with the
+        // one-store scale path below.)
         for (int kt = 0; kt < num_kt; ++kt, ++it) {
           const int stage = static_cast<int>(it % STAGES);
           const uint32_t round = it / STAGES;
-          if (!mbar_wait_cluster(&full[stage], round & 1, kWaitTimeoutNs) ||
-              !mbar_wait_cluster(&sf_full[stage], round & 1, kWaitTimeoutNs)) {
+          if (!mbar_wait_cluster(&full[stage], round & 1, kWaitTimeoutNs)) {
             report_timeout(p.dev_status);
             ok = false;
             break;
           }
           tc_fence_after();
-          if (prev >= 0) tc_commit_pair(&empty[prev], 0x3);
           const int nk64 = min(kK64PerStage, num_k64 - kt * kK64PerStage);
           const uint32_t sA = smem_u32(smem + C::kOffA + stage * C::kABytes);
           const uint32_t sB = smem_u32(smem + C::kOffB + stage * C::kBBytes);
@@ -1203,9 +1215,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
                           slot + kK64PerStage * C::kSfaColsPerK64 + a * C::kSfbColsPerK64,
                           (kt | a) != 0 ? 1u : 0u);
           }
-          prev = stage;
+          tc_commit_pair(&empty[stage], 0x3);
         }
-        if (prev >= 0) tc_commit_pair(&empty[prev], 0x3);
         if (ok) tc_commit_pair(acc_full, 0x3);
       }
     }
@@ -1214,7 +1225,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
     // ------------------------------------------------------------------ scale warps (each CTA)
     const int q = warp & 3;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t sf_full0 = mapa_shared(smem_u32(&sf_full[0]), 0);
+    const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
     uint32_t it = 0;
     bool ok = true;
     for (int t = pair; t < num_tiles && ok; t += npairs) {
@@ -1231,20 +1242,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
         const uint8_t *sSfb = smem + C::kOffSfb + stage * C::kSfbBytes;
         const uint32_t slot = lane_base + C::kSfCol0 + stage * C::kSlotCols;
         const uint32_t slot_b = slot + kK64PerStage * C::kSfaColsPerK64;
-        // same tensor-memory scale layout as the single-CTA kernel with a 256-row B operand
-        for (int a = 0; a < nk64; ++a) {
-          const uint32_t wa =
-              *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
-          tmem_st_x1(slot + a * C::kSfaColsPerK64 + q, wa);  // quarter q reads column base + q
-          const uint4 b0 = *reinterpret_cast<const uint4 *>(sSfb + a * kSfAtomBytes + lane * 16);
-          const uint4 b1 = *reinterpret_cast<const uint4 *>(
-              sSfb + (kK64PerStage + a) * kSfAtomBytes + lane * 16);
-          tmem_st_x8(slot_b + a * C::kSfbColsPerK64, b0, b1);
+        // same tensor-memory scale layout as the single-CTA kernel with a 256-row B operand;
+        // a full stage's B words (four K64 steps x 8 columns) are contiguous columns and go
+        // out in one 32-column store
+        if (nk64 == kK64PerStage) {
+          uint32_t bw[4 * C::kSfbColsPerK64];
+#pragma unroll
+          for (int a = 0; a < kK64PerStage; ++a) {
+            const uint32_t wa =
+                *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
+            tmem_st_x1(slot + a * C::kSfaColsPerK64 + q, wa);  // quarter q reads column base + q
+            const uint4 b0 = *reinterpret_cast<const uint4 *>(sSfb + a * kSfAtomBytes + lane * 16);
+            const uint4 b1 = *reinterpret_cast<const uint4 *>(
+                sSfb + (kK64PerStage + a) * kSfAtomBytes + lane * 16);
+            bw[8 * a + 0] = b0.x; bw[8 * a + 1] = b0.y; bw[8 * a + 2] = b0.z; bw[8 * a + 3] = b0.w;
+            bw[8 * a + 4] = b1.x; bw[8 * a + 5] = b1.y; bw[8 * a + 6] = b1.z; bw[8 * a + 7] = b1.w;
+          }
+          tmem_st_x32(slot_b, bw);
+        } else {
+          for (int a = 0; a < nk64; ++a) {
+            const uint32_t wa =
+                *reinterpret_cast<const uint32_t *>(sSfa + a * kSfAtomBytes + lane * 16 + q * 4);
+            tmem_st_x1(slot + a * C::kSfaColsPerK64 + q, wa);
+            const uint4 b0 = *reinterpret_cast<const uint4 *>(sSfb + a * kSfAtomBytes + lane * 16);
+            const uint4 b1 = *reinterpret_cast<const uint4 *>(
+                sSfb + (kK64PerStage + a) * kSfAtomBytes + lane * 16);
+            tmem_st_x8(slot_b + a * C::kSfbColsPerK64, b0, b1);
+          }
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(sf_full0 + stage * 8);
+        if (lane == 0) mbar_arrive_cluster(full0 + stage * 8);
       }
     }
   } else if (warp >= kEpiWarp0) {
