@@ -1381,7 +1381,8 @@ static EncodeTiledFn encode_fn() {
 }
 
 // 2-D map over a packed [rows, K/2] byte matrix, box = 128 bytes x box_rows, 128-byte swizzle;
-// reads past the last row or column are zero-filled.
+// reads past the last row or column are zero-filled. L2 promotion of 128 bytes (one box row):
+// on B200 the small-M GEMM ran 0.7 % faster than with 256-byte promotion, the prefill GEMM the same.
 static bool encode_operand_map(CUtensorMap *map, const void *base, int64_t rows, int64_t k_bytes,
                                int box_rows) {
   EncodeTiledFn enc = encode_fn();
@@ -1392,7 +1393,7 @@ static bool encode_operand_map(CUtensorMap *map, const void *base, int64_t rows,
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
