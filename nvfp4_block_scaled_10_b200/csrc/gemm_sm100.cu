@@ -689,38 +689,53 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The next kernel in the stream, if it was launched as a programmatic dependent, may start
+  // as this kernel's CTAs leave their SMs; it waits for this kernel to finish before it
+  // touches anything this kernel reads or writes, except the weights.
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (NPL == 1 && p.a_sf_8x4 && lane == 0) {
-      // rows 0..31 of the 8x4 activation scales: four blocks of K/64 x 32 contiguous bytes
-      const uint32_t blk = static_cast<uint32_t>(k64_per_row * 32);
-      const int nblk = static_cast<int>(p.a_sf_rows / 8);
-      mbar_arrive_expect_tx(sfb_ready, blk * nblk);
-      for (int b = 0; b < nblk; ++b)
-        bulk_g2s(smem + C::kOffSfb + b * blk, p.a_sf + static_cast<int64_t>(b) * blk, blk, sfb_ready);
-    }
     uint32_t it = 0;
     bool ok = true;
-    // fp32 scales: the plane words come from the kernel before this one, so the first ring
-    // pass goes out without them (its stages' byte counts include them) and, once that
-    // kernel has finished, their copies follow, before any stage can be reused
-    bool planes_out = NPL == 1;
-    auto issue_first_planes = [&](uint32_t n) {
+    // The activations, their scales and the plane words may come from the kernel before this
+    // one (this kernel is launched as its programmatic dependent), so the first ring pass
+    // streams the weights and their scales only; its stages' byte counts include the rest.
+    // Once that kernel has finished (griddepcontrol.wait) the activation copies of those
+    // stages follow, before any stage is reused.
+    bool first_pass_done = false;
+    auto issue_first_pass_rest = [&](uint32_t n) {
       if (lane == 0) {
         griddep_wait();
+        if (NPL == 1 && p.a_sf_8x4) {
+          // rows 0..31 of the 8x4 activation scales: four blocks of K/64 x 32 contiguous bytes
+          const uint32_t blk = static_cast<uint32_t>(k64_per_row * 32);
+          const int nblk = static_cast<int>(p.a_sf_rows / 8);
+          mbar_arrive_expect_tx(sfb_ready, blk * nblk);
+          for (int b = 0; b < nblk; ++b)
+            bulk_g2s(smem + C::kOffSfb + b * blk, p.a_sf + static_cast<int64_t>(b) * blk, blk, sfb_ready);
+        }
         KStream ks;
         ks.itr = start;
         ks.kt = ks.ke = 0;
         for (uint32_t i = 0; i < n; ++i) {
-          const int k64 = ks.next() * kK64PerStage;
+          const int kt = ks.next();
+          const int k64 = kt * kK64PerStage;
           const int nk = min(kK64PerStage, num_k64 - k64);
-          bulk_g2s(smem + C::kOffSfbStage + i * C::kSfbBytes, p.planes + static_cast<int64_t>(k64) * NPL * 32,
-                   nk * NPL * 128, &full[i]);
+#pragma unroll
+          for (int pl = 0; pl < NPL; ++pl)  // the token tile once per scale plane
+            tma_load_2d(smem + C::kOffB + i * C::kBBytes + pl * (kDecBN * kBKBytes), &tmap_a, kt * kBKBytes,
+                        0, &full[i]);
+          if (NPL > 1)
+            bulk_g2s(smem + C::kOffSfbStage + i * C::kSfbBytes, p.planes + static_cast<int64_t>(k64) * NPL * 32,
+                     nk * NPL * 128, &full[i]);
+          else if (!p.a_sf_8x4)
+            bulk_g2s(smem + C::kOffSfbStage + i * C::kSfbBytes, p.a_sf + static_cast<int64_t>(k64) * kSfAtomBytes,
+                     nk * kSfAtomBytes, &full[i]);
         }
       }
       __syncwarp();
-      planes_out = true;
+      first_pass_done = true;
     };
     DecIter itr = start;
     int tile, kb, ke;
@@ -735,7 +750,7 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
           ok = false;
           break;
         }
-        if (!planes_out && it == STAGES) issue_first_planes(STAGES);
+        if (!first_pass_done && it == STAGES) issue_first_pass_rest(STAGES);
         if (it >= STAGES && !mbar_wait_warp(&empty[stage], (round - 1) & 1, p.wait_ns)) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
@@ -749,27 +764,27 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
           mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes + sf_bytes);
           tma_load_2d(smem + C::kOffA + stage * C::kABytes, &tmap_w, kt * kBKBytes,
                       static_cast<int32_t>(w0), &full[stage]);
-#pragma unroll
-          for (int pl = 0; pl < NPL; ++pl)  // the token tile once per scale plane
-            tma_load_2d(smem + C::kOffB + stage * C::kBBytes + pl * (kDecBN * kBKBytes), &tmap_a,
-                        kt * kBKBytes, 0, &full[stage]);
           bulk_g2s(smem + C::kOffSfa + stage * C::kSfaBytes,
                    p.w_sf + ((w0 / 128) * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
                    &full[stage]);
-          if (NPL > 1) {
-            if (planes_out)
+          if (first_pass_done) {
+#pragma unroll
+            for (int pl = 0; pl < NPL; ++pl)  // the token tile once per scale plane
+              tma_load_2d(smem + C::kOffB + stage * C::kBBytes + pl * (kDecBN * kBKBytes), &tmap_a,
+                          kt * kBKBytes, 0, &full[stage]);
+            if (NPL > 1)
               bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
                        p.planes + static_cast<int64_t>(k64_0) * NPL * 32, nk64 * NPL * 128, &full[stage]);
-          } else if (!p.a_sf_8x4) {  // tokens 0..31: the first 128-row block of the 128x4 scales
-            bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
-                     p.a_sf + static_cast<int64_t>(k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
-                     &full[stage]);
+            else if (!p.a_sf_8x4)  // tokens 0..31: the first 128-row block of the 128x4 scales
+              bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
+                       p.a_sf + static_cast<int64_t>(k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
+                       &full[stage]);
           }
         }
         __syncwarp();
       }
     }
-    if (!planes_out) issue_first_planes(it < STAGES ? it : STAGES);
+    if (!first_pass_done) issue_first_pass_rest(it < STAGES ? it : STAGES);
     if (ok) {
       const uint32_t used = it < STAGES ? it : STAGES;
       for (uint32_t i = 0; i < used; ++i) {
@@ -888,8 +903,10 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     const int q = warp & 3;
     const int row = q * 32 + lane;  // weight row within the tile (accumulator lane)
     float alpha[kDecBN];  // per token (accumulator column)
+    // the row factors and global scales may come from the kernel before this one, and the
+    // output and workspace may still be in use by it
+    griddep_wait();
     if constexpr (NPL > 1) {
-      griddep_wait();  // the row factors come from the kernel before this one
 #pragma unroll
       for (int j = 0; j < kDecBN; ++j) alpha[j] = __ldcg(p.row_alpha + j);
     } else {
@@ -1114,6 +1131,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
   cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The next kernel in the stream, if it was launched as a programmatic dependent, may start
+  // as this kernel's CTAs leave their SMs; it waits for this kernel to finish before it
+  // touches anything this kernel reads or writes, except the weights.
+  griddep_launch_dependents();
 
   auto tile_origin = [&](int t, int64_t &m0, int64_t &n0) {
     m0 = static_cast<int64_t>(t % p.tiles_a) * 256;
@@ -1125,6 +1146,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
     uint32_t it = 0;
     bool ok = true;
     const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
+    // A and its scales may come from the kernel before this one (this kernel is launched as
+    // its programmatic dependent), so the first ring pass loads B (the weights) and B's
+    // scales only; its stages' byte counts include the rest. Once that kernel has finished
+    // (griddepcontrol.wait) the A copies of those stages follow, before any stage is reused.
+    bool first_pass_done = false;
+    auto issue_first_pass_rest = [&](uint32_t n) {
+      if (lane == 0) {
+        griddep_wait();
+        uint32_t i = 0;
+        for (int t = pair; t < num_tiles && i < n; t += npairs) {
+          int64_t m0, n0;
+          tile_origin(t, m0, n0);
+          const int64_t arow = m0 + C::kHalf * rank;
+          for (int kt = 0; kt < num_kt && i < n; ++kt, ++i) {
+            const int k64_0 = kt * kK64PerStage;
+            const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+            if (arow < p.sfa_rows_padded)
+              bulk_g2s(smem + C::kOffSfa + i * C::kSfaBytes,
+                       p.sfa + ((arow / 128) * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
+                       &sf_ready[i]);
+            tma_load_2d_pair(smem + C::kOffA + i * C::kABytes, &tmap_a, kt * kBKBytes,
+                             static_cast<int32_t>(arow), full0 + i * 8);
+          }
+        }
+      }
+      __syncwarp();
+      first_pass_done = true;
+    };
     for (int t = pair; t < num_tiles && ok; t += npairs) {
       int64_t m0, n0;
       tile_origin(t, m0, n0);
@@ -1137,6 +1186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
       for (int kt = 0; kt < num_kt; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
+        if (!first_pass_done && it == STAGES) issue_first_pass_rest(STAGES);
         if (it >= STAGES) {
           if (!mbar_wait_cluster_warp(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
             if (lane == 0) report_timeout(p.dev_status);
@@ -1153,7 +1203,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
         if (lane == 0) {
           const uint32_t sf_bytes = ((sfa_copy ? 1 : 0) + sfb_copies) * nk64 * kSfAtomBytes;
           mbar_arrive_expect_tx(&sf_ready[stage], sf_bytes);
-          if (sfa_copy)
+          if (sfa_copy && first_pass_done)
             bulk_g2s(sSfa, p.sfa + ((arow / 128) * k64_per_row + k64_0) * kSfAtomBytes,
                      nk64 * kSfAtomBytes, &sf_ready[stage]);
           for (int blk = 0; blk < sfb_copies; ++blk) {
@@ -1164,12 +1214,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
           }
           const uint32_t fullc = full0 + stage * 8;
           mbar_arrive_expect_tx_cluster(fullc, C::kABytes + C::kBBytes);
-          tma_load_2d_pair(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(arow), fullc);
+          if (first_pass_done)
+            tma_load_2d_pair(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(arow), fullc);
           tma_load_2d_pair(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(brow), fullc);
         }
         __syncwarp();
       }
     }
+    if (!first_pass_done) issue_first_pass_rest(it < STAGES ? it : STAGES);
     if (ok) {
       const uint32_t used = it < STAGES ? it : STAGES;
       for (uint32_t i = 0; i < used; ++i) {
@@ -1290,6 +1342,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
     const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
     uint8_t *const out_stage = smem + C::kOffOut;
     const bool issuer = e == 0 && lane == 0;
+    // the global scales may come from the kernel before this one, and the output may still be
+    // in use by it
+    griddep_wait();
     uint32_t tile_iter = 0;
     for (int t = pair; t < num_tiles; t += npairs, ++tile_iter) {
       int64_t m0, n0;
@@ -1567,9 +1622,9 @@ static cudaError_t run_pair(const GemmArgs &g, int num_sms, cudaStream_t st) {
   const int resident = resident_pairs<STAGES>();
   if (resident <= 0) return cudaErrorLaunchOutOfResources;
   const int64_t pairs = tiles < resident ? tiles : resident;
-  gemm_nvfp4_pair_kernel<STAGES><<<static_cast<int>(2 * pairs), C::kThreads, C::kSmemBytes, st>>>(
-      ma, mb, mo, p);
-  return cudaGetLastError();
+  // clusters of two (compiled in); a programmatic dependent of the kernel before it
+  return launch_dependent(gemm_nvfp4_pair_kernel<STAGES>, dim3(static_cast<unsigned>(2 * pairs)),
+                          dim3(C::kThreads), C::kSmemBytes, st, ma, mb, mo, p);
 }
 
 // Small-M stream-K layout for a device with num_sms SMs: grid, pieces per tile, workspace.
@@ -1685,11 +1740,8 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
   const int smem = C::smem_bytes(static_cast<int>(g.K / 64), p.a_sf_8x4 != 0);
   e = ensure_smem_attr(gemm_nvfp4_decode_kernel<STAGES, NPL>, smem);
   if (e != cudaSuccess) return e;
-  if constexpr (NPL == 1) {
-    gemm_nvfp4_decode_kernel<STAGES, NPL><<<d.grid, C::kThreads, smem, st>>>(mw, ma, p);
-    return cudaGetLastError();
-  } else {
-    // the split kernel first (one warp per row); the GEMM may start while it runs and waits
+  if constexpr (NPL > 1) {
+    // the split kernel first (one CTA per row); the GEMM may start while it runs and waits
     // for it only where it reads the words and factors (griddepcontrol)
     static_assert(NPL == kActPlanes, "the split kernel writes kActPlanes planes");
     uint8_t *region = static_cast<uint8_t *>(g.workspace) + counter_region(g.workspace_bytes) + d.partial_bytes;
@@ -1699,18 +1751,11 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
     p.row_alpha = row_alpha;
     e = launch_act_scale_planes(g.a_sf32, g.M, g.K, g.w_scale, planes, row_alpha, g.dev_status, st);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(d.grid);
-    cfg.blockDim = dim3(C::kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_nvfp4_decode_kernel<STAGES, NPL>, mw, ma, p);
   }
+  // a programmatic dependent of the kernel before it: the weights of the first ring pass
+  // stream in while that kernel's last CTAs finish
+  return launch_dependent(gemm_nvfp4_decode_kernel<STAGES, NPL>, dim3(d.grid), dim3(C::kThreads), smem, st,
+                          mw, ma, p);
 }
 
 bool gemm_act_f32_supported(int64_t K) { return K / 2 <= (int64_t(1) << 31); }

@@ -26,6 +26,27 @@ struct DebugHooks {
 };
 DebugHooks debug_hooks();
 
+// Launches `kernel` as a programmatic dependent of the work before it in the stream
+// (cudaLaunchAttributeProgrammaticStreamSerialization): it may start while the kernel before
+// it still runs, once that kernel's CTAs have all reached griddepcontrol.launch_dependents
+// or exited, and it waits for that kernel (griddepcontrol.wait) before it touches anything
+// that kernel writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 // quantize.cu
 int *device_error_symbol();
 int global_scale_parts(int64_t M, int64_t K, int num_sms);
