@@ -970,25 +970,22 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
       tc_fence_after();
       float vals[kDecBN];
       const uint32_t t_acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
-#pragma unroll
-      for (int cc = 0; cc < kDecBN; cc += 8) {
-        uint32_t v[8];
-        tmem_ld_32x32b_x8(t_acc + cc, v);
+      static_assert(kDecBN == 32, "one 32-column load per plane");
+      {
+        uint32_t v[kDecBN];
+        tmem_ld_32x32b_x32(t_acc, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) vals[cc + j] = __uint_as_float(v[j]);
+        for (int j = 0; j < kDecBN; ++j) vals[j] = __uint_as_float(v[j]);
       }
       // the planes' partial sums of token j sit in columns j, 32 + j, 64 + j
 #pragma unroll
       for (int pl = 1; pl < NPL; ++pl) {
+        uint32_t v[kDecBN];
+        tmem_ld_32x32b_x32(t_acc + pl * kDecBN, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < kDecBN; cc += 8) {
-          uint32_t v[8];
-          tmem_ld_32x32b_x8(t_acc + pl * kDecBN + cc, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 8; ++j) vals[cc + j] = __fadd_rn(vals[cc + j], __uint_as_float(v[j]));
-        }
+        for (int j = 0; j < kDecBN; ++j) vals[j] = __fadd_rn(vals[j], __uint_as_float(v[j]));
       }
       tc_fence_before();
       __syncwarp();
