@@ -338,8 +338,8 @@ def run_ours(args, rank, world, torch, dist):
         out = torch.empty(M, N, dtype=torch.float16, device=dev)
         alg = algorithmic(wl, M=M, N=N, K=K, a_layout=args.a_layout)
         kernel_key = f"gemm_{wl}"
-        kernel_name = {"decode": "gemm_nvfp4_decode_kernel<7,1>", "decode_f32": "gemm_nvfp4_decode_kernel<7,3>",
-                       "prefill": "gemm_nvfp4_pair_kernel<5>"}.get(wl, "gemm_nvfp4_kernel")
+        kernel_name = {"decode": "gemm_nvfp4_decode_kernel<5,1>", "decode_f32": "gemm_nvfp4_decode_kernel<5,3>",
+                       "prefill": "gemm_nvfp4_pair_kernel<4>"}.get(wl, "gemm_nvfp4_kernel")
 
         if wl == "decode_f32":
             ws_bytes = nv.nvfp4_gemm_act_f32_workspace_bytes(M, N, K)

@@ -8,7 +8,10 @@
  *    the fixed library array of nvfp4_global_scale_noalloc). Sizes are element counts
  *    unless stated.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Calls
- *    are asynchronous on that stream and return once the work is enqueued.
+ *    are asynchronous on that stream and return once the work is enqueued. The GEMM kernels
+ *    are launched as programmatic dependents of the kernel before them on the stream: they
+ *    may start while it finishes, but until it has completed they only prefetch weights
+ *    into L2, so every call keeps plain stream order (any earlier work may write any input).
  *  - Return value: an nvfp4_status. Argument errors are detected on the host before any
  *    launch and nothing is enqueued. NVFP4_ERR_CUDA reports a launch error
  *    (cudaGetLastError after the launch). Errors raised later by a kernel surface on the

@@ -694,8 +694,8 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // The next kernel in the stream, if it was launched as a programmatic dependent, may start
-  // as this kernel's CTAs leave their SMs; it waits for this kernel to finish before it
-  // touches anything this kernel reads or writes, except the weights.
+  // as this kernel's CTAs leave their SMs; the GEMM kernels here only prefetch into L2 until
+  // this kernel has finished.
   griddep_launch_dependents();
 
   if (warp == 0) {
@@ -704,45 +704,35 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     bool ok = true;
     // Each stage has two barriers: sf_loaded[s] for the scale words (the scale warps start on
     // them as soon as they land) and full[s] for the weight and token tiles (the MMA thread).
-    // The activations, their scales and the plane words may come from the kernel before this
-    // one (this kernel is launched as its programmatic dependent), so the first ring pass
-    // streams the weights and their scales only; its stages' byte counts include the rest.
-    // Once that kernel has finished (griddepcontrol.wait) the activation copies of those
-    // stages follow, before any stage is reused.
-    bool first_pass_done = false;
-    auto issue_first_pass_rest = [&](uint32_t n) {
-      if (lane == 0) {
-        griddep_wait();
-        if (NPL == 1 && p.a_sf_8x4) {
-          // rows 0..31 of the 8x4 activation scales: four blocks of K/64 x 32 contiguous bytes
-          const uint32_t blk = static_cast<uint32_t>(k64_per_row * 32);
-          const int nblk = static_cast<int>(p.a_sf_rows / 8);
-          mbar_arrive_expect_tx(sfb_ready, blk * nblk);
-          for (int b = 0; b < nblk; ++b)
-            bulk_g2s(smem + C::kOffSfb + b * blk, p.a_sf + static_cast<int64_t>(b) * blk, blk, sfb_ready);
-        }
-        KStream ks;
-        ks.itr = start;
-        ks.kt = ks.ke = 0;
-        for (uint32_t i = 0; i < n; ++i) {
-          const int kt = ks.next();
-          const int k64 = kt * kK64PerStage;
-          const int nk = min(kK64PerStage, num_k64 - k64);
-#pragma unroll
-          for (int pl = 0; pl < NPL; ++pl)  // the token tile once per scale plane
-            tma_load_2d(smem + C::kOffB + i * C::kBBytes + pl * (kDecBN * kBKBytes), &tmap_a, kt * kBKBytes,
-                        0, &full[i]);
-          if (NPL > 1)
-            bulk_g2s(smem + C::kOffSfbStage + i * C::kSfbBytes, p.planes + static_cast<int64_t>(k64) * NPL * 32,
-                     nk * NPL * 128, &sf_loaded[i]);
-          else if (!p.a_sf_8x4)
-            bulk_g2s(smem + C::kOffSfbStage + i * C::kSfbBytes, p.a_sf + static_cast<int64_t>(k64) * kSfAtomBytes,
-                     nk * kSfAtomBytes, &sf_loaded[i]);
+    // This kernel is launched as a programmatic dependent of the kernel before it: while that
+    // kernel finishes, the weights and weight scales of the first ring pass are prefetched
+    // into L2 (no shared-memory write, nothing read before it is complete), and every copy
+    // into shared memory waits for it (griddepcontrol.wait), so the kernel before may write
+    // any of this call's inputs.
+    if (lane == 0) {
+      DecIter pit = start;
+      int tile, kb, ke;
+      int n = 0;
+      while (n < STAGES && pit.next(tile, kb, ke)) {
+        for (int kt = kb; kt < ke && n < STAGES; ++kt, ++n) {
+          const int k64_0 = kt * kK64PerStage;
+          const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+          tma_prefetch_l2_2d(&tmap_w, kt * kBKBytes, tile * kBM);
+          bulk_prefetch_l2(p.w_sf + (static_cast<int64_t>(tile) * k64_per_row + k64_0) * kSfAtomBytes,
+                           nk64 * kSfAtomBytes);
         }
       }
-      __syncwarp();
-      first_pass_done = true;
-    };
+      griddep_wait();
+      if (NPL == 1 && p.a_sf_8x4) {
+        // rows 0..31 of the 8x4 activation scales: four blocks of K/64 x 32 contiguous bytes
+        const uint32_t blk = static_cast<uint32_t>(k64_per_row * 32);
+        const int nblk = static_cast<int>(p.a_sf_rows / 8);
+        mbar_arrive_expect_tx(sfb_ready, blk * nblk);
+        for (int b = 0; b < nblk; ++b)
+          bulk_g2s(smem + C::kOffSfb + b * blk, p.a_sf + static_cast<int64_t>(b) * blk, blk, sfb_ready);
+      }
+    }
+    __syncwarp();
     DecIter itr = start;
     int tile, kb, ke;
     while (ok && itr.next(tile, kb, ke)) {
@@ -756,7 +746,6 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
           ok = false;
           break;
         }
-        if (!first_pass_done && it == STAGES) issue_first_pass_rest(STAGES);
         if (it >= STAGES && !mbar_wait_warp(&empty[stage], (round - 1) & 1, p.wait_ns)) {
           if (lane == 0) report_timeout(p.dev_status);
           ok = false;
@@ -771,29 +760,24 @@ __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
           bulk_g2s(smem + C::kOffSfa + stage * C::kSfaBytes,
                    p.w_sf + ((w0 / 128) * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
                    &sf_loaded[stage]);
-          if (first_pass_done) {
-            if (NPL > 1)
-              bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
-                       p.planes + static_cast<int64_t>(k64_0) * NPL * 32, nk64 * NPL * 128, &sf_loaded[stage]);
-            else if (!p.a_sf_8x4)  // tokens 0..31: the first 128-row block of the 128x4 scales
-              bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
-                       p.a_sf + static_cast<int64_t>(k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
-                       &sf_loaded[stage]);
-          }
+          if (NPL > 1)
+            bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
+                     p.planes + static_cast<int64_t>(k64_0) * NPL * 32, nk64 * NPL * 128, &sf_loaded[stage]);
+          else if (!p.a_sf_8x4)  // tokens 0..31: the first 128-row block of the 128x4 scales
+            bulk_g2s(smem + C::kOffSfbStage + stage * C::kSfbBytes,
+                     p.a_sf + static_cast<int64_t>(k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
+                     &sf_loaded[stage]);
           mbar_arrive_expect_tx(&full[stage], C::kABytes + C::kBBytes);
           tma_load_2d(smem + C::kOffA + stage * C::kABytes, &tmap_w, kt * kBKBytes,
                       static_cast<int32_t>(w0), &full[stage]);
-          if (first_pass_done) {
 #pragma unroll
-            for (int pl = 0; pl < NPL; ++pl)  // the token tile once per scale plane
-              tma_load_2d(smem + C::kOffB + stage * C::kBBytes + pl * (kDecBN * kBKBytes), &tmap_a,
-                          kt * kBKBytes, 0, &full[stage]);
-          }
+          for (int pl = 0; pl < NPL; ++pl)  // the token tile once per scale plane
+            tma_load_2d(smem + C::kOffB + stage * C::kBBytes + pl * (kDecBN * kBKBytes), &tmap_a,
+                        kt * kBKBytes, 0, &full[stage]);
         }
         __syncwarp();
       }
     }
-    if (!first_pass_done) issue_first_pass_rest(it < STAGES ? it : STAGES);
     if (ok) {
       const uint32_t used = it < STAGES ? it : STAGES;
       for (uint32_t i = 0; i < used; ++i) {
@@ -1171,8 +1155,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // The next kernel in the stream, if it was launched as a programmatic dependent, may start
-  // as this kernel's CTAs leave their SMs; it waits for this kernel to finish before it
-  // touches anything this kernel reads or writes, except the weights.
+  // as this kernel's CTAs leave their SMs; the GEMM kernels here only prefetch into L2 until
+  // this kernel has finished.
   griddep_launch_dependents();
 
   auto tile_origin = [&](int t, int64_t &m0, int64_t &n0) {
@@ -1185,34 +1169,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
     uint32_t it = 0;
     bool ok = true;
     const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);
-    // A and its scales may come from the kernel before this one (this kernel is launched as
-    // its programmatic dependent), so the first ring pass loads B (the weights) and B's
-    // scales only; its stages' byte counts include the rest. Once that kernel has finished
-    // (griddepcontrol.wait) the A copies of those stages follow, before any stage is reused.
-    bool first_pass_done = false;
-    auto issue_first_pass_rest = [&](uint32_t n) {
-      if (lane == 0) {
-        griddep_wait();
-        uint32_t i = 0;
-        for (int t = pair; t < num_tiles && i < n; t += npairs) {
-          int64_t m0, n0;
-          tile_origin(t, m0, n0);
-          const int64_t arow = m0 + C::kHalf * rank;
-          for (int kt = 0; kt < num_kt && i < n; ++kt, ++i) {
-            const int k64_0 = kt * kK64PerStage;
-            const int nk64 = min(kK64PerStage, num_k64 - k64_0);
-            if (arow < p.sfa_rows_padded)
-              bulk_g2s(smem + C::kOffSfa + i * C::kSfaBytes,
-                       p.sfa + ((arow / 128) * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes,
-                       &sf_ready[i]);
-            tma_load_2d_pair(smem + C::kOffA + i * C::kABytes, &tmap_a, kt * kBKBytes,
-                             static_cast<int32_t>(arow), full0 + i * 8);
+    // This kernel is launched as a programmatic dependent of the kernel before it: while that
+    // kernel finishes, this CTA's B rows (the weights) and B's scale atoms for the first ring
+    // pass are prefetched into L2 (no shared-memory write, nothing read before it is
+    // complete), and every copy into shared memory waits for it (griddepcontrol.wait), so the
+    // kernel before may write any of this call's inputs.
+    if (lane == 0) {
+      int n = 0;
+      for (int t = pair; t < num_tiles && n < STAGES; t += npairs) {
+        int64_t m0, n0;
+        tile_origin(t, m0, n0);
+        const int64_t brow = n0 + C::kHalf * rank;
+        for (int kt = 0; kt < num_kt && n < STAGES; ++kt, ++n) {
+          const int k64_0 = kt * kK64PerStage;
+          const int nk64 = min(kK64PerStage, num_k64 - k64_0);
+          tma_prefetch_l2_2d(&tmap_b, kt * kBKBytes, static_cast<int32_t>(brow));
+          for (int blk = 0; blk < 2; ++blk) {
+            const int64_t rb = n0 / 128 + blk;
+            if (rb * 128 < p.sfb_rows_padded)
+              bulk_prefetch_l2(p.sfb + (rb * k64_per_row + k64_0) * kSfAtomBytes, nk64 * kSfAtomBytes);
           }
         }
       }
-      __syncwarp();
-      first_pass_done = true;
-    };
+      griddep_wait();
+    }
+    __syncwarp();
     for (int t = pair; t < num_tiles && ok; t += npairs) {
       int64_t m0, n0;
       tile_origin(t, m0, n0);
@@ -1225,7 +1206,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
       for (int kt = 0; kt < num_kt; ++kt, ++it) {
         const int stage = static_cast<int>(it % STAGES);
         const uint32_t round = it / STAGES;
-        if (!first_pass_done && it == STAGES) issue_first_pass_rest(STAGES);
         if (it >= STAGES) {
           if (!mbar_wait_cluster_warp(&empty[stage], (round - 1) & 1, kWaitTimeoutNs)) {
             if (lane == 0) report_timeout(p.dev_status);
@@ -1242,7 +1222,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
         if (lane == 0) {
           const uint32_t sf_bytes = ((sfa_copy ? 1 : 0) + sfb_copies) * nk64 * kSfAtomBytes;
           mbar_arrive_expect_tx(&sf_ready[stage], sf_bytes);
-          if (sfa_copy && first_pass_done)
+          if (sfa_copy)
             bulk_g2s(sSfa, p.sfa + ((arow / 128) * k64_per_row + k64_0) * kSfAtomBytes,
                      nk64 * kSfAtomBytes, &sf_ready[stage]);
           for (int blk = 0; blk < sfb_copies; ++blk) {
@@ -1253,14 +1233,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<STAGES>::kTh
           }
           const uint32_t fullc = full0 + stage * 8;
           mbar_arrive_expect_tx_cluster(fullc, C::kABytes + C::kBBytes);
-          if (first_pass_done)
-            tma_load_2d_pair(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(arow), fullc);
+          tma_load_2d_pair(sA, &tmap_a, kt * kBKBytes, static_cast<int32_t>(arow), fullc);
           tma_load_2d_pair(sB, &tmap_b, kt * kBKBytes, static_cast<int32_t>(brow), fullc);
         }
         __syncwarp();
       }
     }
-    if (!first_pass_done) issue_first_pass_rest(it < STAGES ? it : STAGES);
     if (ok) {
       const uint32_t used = it < STAGES ? it : STAGES;
       for (uint32_t i = 0; i < used; ++i) {
@@ -1791,8 +1769,8 @@ static cudaError_t run_decode(const GemmArgs &g, const DecPlan &d, cudaStream_t 
     e = launch_act_scale_planes(g.a_sf32, g.M, g.K, g.w_scale, planes, row_alpha, g.dev_status, st);
     if (e != cudaSuccess) return e;
   }
-  // a programmatic dependent of the kernel before it: the weights of the first ring pass
-  // stream in while that kernel's last CTAs finish
+  // a programmatic dependent of the kernel before it: the weights of the first ring pass are
+  // prefetched into L2 while that kernel's last CTAs finish
   return launch_dependent(gemm_nvfp4_decode_kernel<STAGES, NPL>, dim3(d.grid), dim3(C::kThreads), smem, st,
                           mw, ma, p);
 }
@@ -1811,7 +1789,9 @@ cudaError_t launch_gemm_act_f32(const GemmArgs &g, int num_sms, cudaStream_t st)
     c.out = static_cast<__half *>(g.out) + m0 * g.N;
     const DecPlan d = dec_plan(c.M, g.N, g.K, num_sms);
     if (!d.usable) return cudaErrorNotSupported;
-    const cudaError_t e = run_decode<7, kActPlanes>(c, d, st);
+    // 5 stages of 31.5 KB: 34.9 us per call (split kernel included) at M = 32, N = 28672,
+    // K = 8192 on B200, against 35.1 (6 stages) and 36.3 (7)
+    const cudaError_t e = run_decode<5, kActPlanes>(c, d, st);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -29,8 +29,8 @@ DebugHooks debug_hooks();
 // Launches `kernel` as a programmatic dependent of the work before it in the stream
 // (cudaLaunchAttributeProgrammaticStreamSerialization): it may start while the kernel before
 // it still runs, once that kernel's CTAs have all reached griddepcontrol.launch_dependents
-// or exited, and it waits for that kernel (griddepcontrol.wait) before it touches anything
-// that kernel writes or reads.
+// or exited. Until it has waited for that kernel (griddepcontrol.wait) it may only prefetch
+// into L2: no load into shared memory or registers, no write.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                              Args &&...args) {

@@ -2,8 +2,8 @@
 
 The GEMM kernels (the small-M stream-K kernel and the CTA-pair kernel) are launched as
 programmatic dependents of the kernel before them: they may start while that kernel
-finishes, stream the weights of their first ring pass, and wait for it
-(griddepcontrol.wait) before they read what it wrote or write what it reads. Each chain here has calls that read the previous call's output, share
+finishes and prefetch the weights of their first ring pass into L2, and they wait for it
+(griddepcontrol.wait) before any load of an input or any write. Each chain here has calls that read the previous call's output, share
 one workspace, or rewrite a buffer the previous call used. Every result must equal, bit for
 bit, the result of the same call made alone between two synchronisations (the kernels are
 deterministic), eagerly and replayed from a CUDA graph; the alone results of the first link
@@ -202,6 +202,39 @@ def test_gemm_after_torch_writer():
         torch.bitwise_xor(sf, 0, out=sf_buf)
         torch.mul(g, 1.0, out=g_buf)
         got.append(nv.nvfp4_gemm(q_buf, sf_buf, g_buf, wq, wsf, gw, workspace=ws))
+    torch.cuda.synchronize()
+    for i, out in enumerate(got):
+        np.testing.assert_array_equal(host_bytes(out), want[i], err_msg=f"call {i}")
+
+
+@pytest.mark.parametrize("M", [32, 512])
+def test_gemm_after_weight_writer(M):
+    """The weights rewritten on the GPU by the quantize kernel right before each call (the
+    GEMM prefetches its first weight tiles while that kernel may still run)."""
+    nv = require_cuda()
+    N, K = 1280, 2048
+    xb = workloads.bits16(workloads.normal((M, K), seed=900 + M))
+    ga = orc.global_scale(xb)
+    aq, asf, _ = orc.quantize(xb, g=ga)
+    a_dev = (torch.from_numpy(aq).cuda(), torch.from_numpy(orc.swizzle(asf, orc.L128x4)).cuda(),
+             torch.tensor([ga], dtype=torch.float32, device="cuda"))
+    ws_ = [workloads.normal((N, K), std=0.05, seed=910 + i).cuda() for i in range(4)]
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device="cuda")
+    wsf = torch.empty(nv.nvfp4_sf_bytes(N, K), dtype=torch.uint8, device="cuda")
+    gw = torch.empty(1, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(max(nv.nvfp4_gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device="cuda")
+    want = []
+    for w in ws_:
+        nv.nvfp4_global_scale(w, gw)
+        nv.nvfp4_quantize(w, gw, q=wq, sf=wsf)
+        torch.cuda.synchronize()
+        want.append(host_bytes(nv.nvfp4_gemm(*a_dev, wq, wsf, gw, workspace=ws)))
+        torch.cuda.synchronize()
+    got = []
+    for w in ws_:
+        nv.nvfp4_global_scale(w, gw)
+        nv.nvfp4_quantize(w, gw, q=wq, sf=wsf)
+        got.append(nv.nvfp4_gemm(*a_dev, wq, wsf, gw, workspace=ws))
     torch.cuda.synchronize()
     for i, out in enumerate(got):
         np.testing.assert_array_equal(host_bytes(out), want[i], err_msg=f"call {i}")
