@@ -620,20 +620,6 @@ __device__ __forceinline__ bool group_all(bool v, int id, int nthreads) {
 __device__ __forceinline__ bool epi_all(bool v, int nthreads) { return group_all(v, 1, nthreads); }
 
 
-// The K-steps a CTA walks, one by one, in its segments' order (-1 once they run out).
-struct KStream {
-  DecIter itr;
-  int kt, ke;
-  __device__ __forceinline__ int next() {
-    if (kt >= ke) {
-      int tile, kb;
-      if (!itr.next(tile, kb, ke)) return -1;
-      kt = kb;
-    }
-    return kt++;
-  }
-};
-
 template <int STAGES, int NPL>
 __global__ void __launch_bounds__(DecCfg<STAGES, NPL>::kThreads, 1)
     gemm_nvfp4_decode_kernel(const __grid_constant__ CUtensorMap tmap_w,
